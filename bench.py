@@ -1,0 +1,411 @@
+"""Benchmark of SparSTAR's per-scale block-sparse attention forward.
+
+One step = the whole path for one scale of the 72,000-token workload
+(H = 16, D = 128, bf16, density 0.09375): pool Q, pool K, score, select,
+attention, each a launch of libsparstar through its C ABI on one stream,
+with the inputs resident in HBM.  The metric is effective TFLOP/s over the
+selected tiles (algorithmic attention FLOPs = 4 * D * sum over selected
+(query block, key block) pairs of valid queries x valid keys) per step time.
+
+Multi-GPU: the path has no exchange step; ``--gpus N`` runs N independent
+replicas (one process per GPU, launched by torch.distributed.run), timing is
+the max over ranks, and the value is the work of all ranks over that time.
+
+``--impl reference`` times the CPU oracle instead (the comparison arm): each
+step is a bounded sample of the same workload (one head's selection and a
+set of its query rows in fp64), projected to the full step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from datetime import timedelta
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from block_sparse_attention_18_b200 import synth  # noqa: E402
+
+METRIC = "sparse-attn fwd ms + TFLOP/s at 72k-token scale; % of bf16 TC peak"
+UNIT = "TFLOP/s"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic of one attention launch on the benchmark workload, from an
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the
+# SHA-256 of the kernel source it was taken on; reported only while the
+# source is unchanged.
+ATTN_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None}
+
+
+def attn_source_sha256() -> str:
+    path = os.path.join(ROOT, "block_sparse_attention_18_b200", "csrc", "attn_sm100.cu")
+    with open(path, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attention_flops(kv_idx: np.ndarray, kv_cnt: np.ndarray, Lq: int, Lk: int, D: int) -> float:
+    """4 * D * sum over the listed tiles of valid query rows x valid keys."""
+    B, H, nQB, max_sel = kv_idx.shape
+    nKB = (Lk + 127) // 128
+    vq = np.minimum(128, Lq - 128 * np.arange(nQB)).astype(np.float64)
+    vk = np.minimum(128, Lk - 128 * np.arange(nKB)).astype(np.float64)
+    slot = np.arange(max_sel)[None, None, None, :] < kv_cnt[..., None]
+    ok = slot & (kv_idx >= 0) & (kv_idx < nKB)
+    keys = np.where(ok, vk[np.clip(kv_idx, 0, nKB - 1)], 0.0).sum(axis=-1)  # [B,H,nQB]
+    return float(4.0 * D * (keys * vq[None, None, :]).sum())
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def _gpu_id(self):
+        try:
+            uuid = torch.cuda.get_device_properties(self.dev).uuid
+            return "GPU-%s" % uuid
+        except Exception:
+            return str(self.dev)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self._gpu_id(), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [s for s in sm if s > 0.5 * (mx or max(sm))] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (n_gpus, world))
+    if world > 1:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world: int, device):
+    if world > 1:
+        if torch.distributed.get_backend() == "nccl":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Max of a float over ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return value
+    dev = device if torch.distributed.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_sample_step(orc, w, qn, kn, vn, head: int, n_rows: int, seed: int) -> float:
+    """Time the oracle on a bounded sample of one step: the fp32 selection
+    of one head (pool Q, pool K, score, select) and fp64 attention on
+    ``n_rows`` of that head's query rows.  Returns the projected time of a
+    full step in seconds (selection x heads, attention x rows / n_rows)."""
+    sl = slice(head, head + 1)
+    qh = np.ascontiguousarray(qn[:, sl])
+    kh = np.ascontiguousarray(kn[:, sl])
+    vh = np.ascontiguousarray(vn[:, sl])
+    t0 = time.perf_counter()
+    _, _, _, idx, cnt = orc.run_selection(qh, kh, w.text, w.image_ref, w.density)
+    t_sel = time.perf_counter() - t0
+    rows = np.sort(np.random.default_rng(seed).choice(w.Lq, size=min(n_rows, w.Lq), replace=False))
+    t1 = time.perf_counter()
+    orc.attn_rows_f64(qh, kh, vh, idx, cnt, rows.astype(np.int64))
+    t_att = time.perf_counter() - t1
+    heads = w.B * w.H
+    return heads * (t_sel + t_att * (w.Lq / len(rows)))
+
+
+def oracle_flops(orc, w, qn, kn) -> float:
+    """Algorithmic FLOPs of one full step from the oracle's own selection."""
+    _, _, _, idx, cnt = orc.run_selection(qn, kn, w.text, w.image_ref, w.density)
+    return attention_flops(idx, cnt, w.Lq, w.Lk, w.D)
+
+
+def cpu_baseline(w, qn, kn, vn, flops_step: float, budget_s: float = 12.0, n_rows: int = 1024):
+    """The oracle, as it stands, on this host's cores, on a bounded sample."""
+    import oracle as orc
+    orc.lib()
+    t_start = time.perf_counter()
+    times, heads = [], []
+    h = 0
+    while len(times) < 2 or (time.perf_counter() - t_start < budget_s and h < w.B * w.H):
+        times.append(oracle_sample_step(orc, w, qn, kn, vn, h, n_rows, seed=h))
+        heads.append(h)
+        h += 1
+    step_s = statistics.mean(times)
+    return {"value": flops_step / step_s / 1e12, "unit": UNIT, "cores": orc.num_threads(),
+            "kind": "oracle",
+            "sample": ("fp32 selection of heads %s and fp64 attention on %d random query rows of "
+                       "each; time projected to the full step (x%d heads, x%d/%d rows): %.1f s "
+                       "per full step" % (heads, n_rows, w.B * w.H, w.Lq, n_rows, step_s)),
+            "wall_s": time.perf_counter() - t_start}
+
+
+def run_reference(args, world, rank):
+    """The comparison arm: the CPU oracle timed on this host's cores."""
+    if rank != 0:
+        return
+    import oracle as orc
+    orc.lib()
+    w = synth.WORKLOADS[args.workload]
+    q, k, v = synth.generate(w)
+    qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
+    flops = oracle_flops(orc, w, qn, kn)
+    n_rows = args.ref_rows
+    for s in range(args.warmup):
+        oracle_sample_step(orc, w, qn, kn, vn, s % (w.B * w.H), n_rows, seed=1000 + s)
+    times = [oracle_sample_step(orc, w, qn, kn, vn, s % (w.B * w.H), n_rows, seed=s)
+             for s in range(args.steps)]
+    step_s = statistics.mean(times)
+    value = flops / step_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle",
+                         "cores": orc.num_threads(),
+                         "sample": "each step: fp32 selection of one head and fp64 attention on "
+                                   "%d random query rows of it, projected to the full step "
+                                   "(x%d heads, x%d/%d rows)" % (n_rows, w.B * w.H, w.Lq, n_rows)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, world):
+    return {"workload": "%s: H=%d D=%d %s, keys text %d + image_ref %d + ref %d + cur %d = %d, "
+                        "queries %d, density %g" % (w.name, w.H, w.D, w.dtype, w.text, w.image_ref,
+                                                    w.ref, w.cur, w.Lk, w.Lq, w.density),
+            "seq_len": w.Lq, "keys": w.Lk, "heads": w.H, "head_dim": w.D, "density": w.density,
+            "global_batch": w.B * world, "parallelism": "replicas" if world > 1 else "single",
+            "l2": "no flush: inputs (%.2f GB) larger than L2" % (
+                (w.Lq + 2 * w.Lk) * w.H * w.D * (2 if w.dtype == "bf16" else 4) / 1e9)}
+
+
+# --------------------------------------------------------------- GPU arm
+
+def run_gpu(args, world, rank, local):
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    from block_sparse_attention_18_b200 import sparstar as sp
+
+    w = synth.WORKLOADS[args.workload]
+    q, k, v = synth.generate(w)
+    qd, kd, vd = q.to(device), k.to(device), v.to(device)
+    ws = sp.Workspace(w.B, w.H, w.D, w.text, w.image_ref, w.ref, w.cur, w.density, device)
+    out = torch.empty_like(qd)
+    lse = torch.empty(w.B, w.H, w.Lq, device=device, dtype=torch.float32)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    tau = sp.default_tau(w.D)
+    stream = torch.cuda.current_stream(device)
+    names = ["pool_q", "pool_k", "score", "select", "attn"]
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        sp.sparstar_block_pool(qd, ws.qbar, stream=stream)
+        if ev: ev[1].record(stream)
+        sp.sparstar_block_pool(kd, ws.kbar, stream=stream)
+        if ev: ev[2].record(stream)
+        sp.sparstar_block_score(ws.qbar, ws.kbar, tau, ws.S, stream=stream)
+        if ev: ev[3].record(stream)
+        sp.sparstar_select(ws.S, ws.n_forced, w.density, kv_idx=ws.kv_idx, kv_cnt=ws.kv_cnt,
+                           stream=stream)
+        if ev: ev[4].record(stream)
+        sp.sparstar_attn_fwd(qd, kd, vd, ws.kv_idx, ws.kv_cnt, tau, out, lse, status,
+                             stream=stream)
+        if ev: ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if int(status.item()) != 0:
+        raise SystemExit("attention kernel status %#x" % int(status.item()))
+    flops = attention_flops(ws.kv_idx.cpu().numpy(), ws.kv_cnt.cpu().numpy(), w.Lq, w.Lk, w.D)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world, device)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+    ms_per_step = total_ms / args.steps
+    per = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
+           for i, n in enumerate(names)}
+    if int(status.item()) != 0:
+        raise SystemExit("attention kernel status %#x" % int(status.item()))
+
+    # end to end through the C ABI from pinned host buffers
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(args.steps):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        sp.sparstar_forward(qd, kd, vd, w.text, w.image_ref, w.ref, w.cur, w.density,
+                            workspace=ws, out=out, lse=lse, status=status, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world, device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / args.steps
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = out_h.numel() * out_h.element_size()
+
+    if rank != 0:
+        return
+    peaks, peaks_src = read_peaks()
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    attn_tflops = flops / (per["attn"] * 1e-3) / 1e12
+    esz = 2 if w.dtype == "bf16" else 4
+    pool_bytes = ((w.Lq + w.Lk) * w.D * esz + (w.nQB + w.nKB) * w.D * 4) * w.B * w.H
+    score_bytes = ((w.nQB + w.nKB) * w.D * 4 + w.nQB * w.nKB * 4) * w.B * w.H
+    ps_ms = per["pool_q"] + per["pool_k"] + per["score"]
+    ps_gbs = (pool_bytes + score_bytes) / (ps_ms * 1e-3) / 1e9
+    traffic = None
+    if ATTN_TRAFFIC["source_sha256"] == attn_source_sha256():
+        traffic = ATTN_TRAFFIC["bytes_per_launch"]
+    sel_ms = per["pool_q"] + per["pool_k"] + per["score"] + per["select"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, world),
+        "attn_ms": per["attn"], "attn_tflops": attn_tflops,
+        "attn_pct_of_bf16_peak": {"measured_burst": 100 * attn_tflops / peaks["bf16_tflops"],
+                                  "datasheet_2250": 100 * attn_tflops / DATASHEET_BF16_TFLOPS},
+        "kernel_ms": per, "selection_share_pct": 100 * sel_ms / sum(per.values()),
+        "pool_score": {"ms": ps_ms, "gbs": ps_gbs, "frac_of_hbm": ps_gbs / peaks["hbm_gbs"]},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
+                     "traffic": traffic,
+                     "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks_src},
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk.summary(),
+        "flops_per_step_per_gpu": flops,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
+        line["cpu_baseline"] = cpu_baseline(w, qn, kn, vn, flops)
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=list(synth.WORKLOADS))
+    ap.add_argument("--ref-rows", type=int, default=256,
+                    help="query rows per sampled step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,39 @@
+// Internal launch interface between the C ABI layer (sparstar_api.cu) and
+// the kernels.  Not installed; the public interface is include/sparstar.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sparstar {
+
+constexpr int kBlock = 128;  // tokens per block (query and key grids)
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Step 1: block means, fixed fp32 order.  x is bf16 (dtype 0) or fp32 (1).
+cudaError_t launch_pool(const void *x, int dtype, int64_t BH, int64_t L, int D, float *xbar,
+                        cudaStream_t stream);
+
+// Step 2a: S = fl(tau * sequential-fma dot) for every block pair.
+cudaError_t launch_score(const float *qbar, const float *kbar, int64_t BH, int64_t nQB,
+                         int64_t nKB, int D, float tau, float *S, cudaStream_t stream);
+
+// Step 2b: per-row clip-aware top-k into kv_idx / kv_cnt.
+cudaError_t launch_select(const float *S, int64_t rows, int64_t nKB, int64_t nF, int64_t k,
+                          int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel,
+                          cudaStream_t stream);
+
+// Step 3, bf16 D=128: TMA + tcgen05 + TMEM kernel (sm_100a).
+int launch_attn_sm100(const void *q, const void *k, const void *v, int64_t BH, int64_t Lq,
+                      int64_t Lk, float tau, const int32_t *kv_idx, const int32_t *kv_cnt,
+                      int64_t max_sel, void *out, float *lse, int32_t *status,
+                      cudaStream_t stream);
+
+// Step 3, fp32 inputs (D 64/128) and bf16 D=64: fp32 SIMT kernel.
+cudaError_t launch_attn_simt(const void *q, const void *k, const void *v, int dtype,
+                             int64_t BH, int64_t Lq, int64_t Lk, int D, float tau,
+                             const int32_t *kv_idx, const int32_t *kv_cnt, int64_t max_sel,
+                             void *out, float *lse, int32_t *status, cudaStream_t stream);
+
+}  // namespace sparstar

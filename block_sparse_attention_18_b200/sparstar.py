@@ -1,0 +1,207 @@
+"""Python binding of libsparstar (C ABI in include/sparstar.h).
+
+Argument marshalling only: every function reads device pointers, shapes and
+the current CUDA stream from torch tensors, allocates missing outputs with
+torch, and calls the entry point of the same name.  Every step of the path
+runs in the library's kernels; there is no Python or CPU path.  Importing
+this module fails when the library has not been built.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparstar.so")
+BLOCK = 128
+
+OK, EINVAL, EDTYPE, ECUDA, ESIZE, ENODEV = range(6)
+STATUS_BAD_INDEX = 0x1
+STATUS_TIMEOUT = 0x2
+
+_DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libsparstar.so is not built (run block_sparse_attention_18_b200/build.py "
+                          "or __graft_entry__.build()); there is no fallback path")
+    L = ctypes.CDLL(LIB_PATH)
+    i64, i32, f32, f64, vp = (ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_double,
+                              ctypes.c_void_p)
+    L.sparstar_block_pool.argtypes = [vp, i32, i64, i64, i64, i64, vp, vp]
+    L.sparstar_block_score.argtypes = [vp, vp, i64, i64, i64, i64, i64, f32, vp, vp]
+    L.sparstar_forced_blocks.argtypes = [i64, i64]
+    L.sparstar_forced_blocks.restype = i64
+    L.sparstar_select_count.argtypes = [i64, i64, f64]
+    L.sparstar_select_count.restype = i64
+    L.sparstar_select.argtypes = [vp, i64, i64, i64, i64, i64, f64, vp, vp, i64, vp]
+    L.sparstar_attn_fwd.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, f32, vp, vp, i64,
+                                    vp, vp, vp, vp]
+    L.sparstar_forward.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, f64, vp,
+                                   vp, vp, vp, vp, i64, vp, vp, vp, vp]
+    L.sparstar_strerror.argtypes = [i32]
+    L.sparstar_strerror.restype = ctypes.c_char_p
+    L.sparstar_version.restype = i32
+    for name in ("sparstar_block_pool", "sparstar_block_score", "sparstar_select",
+                 "sparstar_attn_fwd", "sparstar_forward"):
+        getattr(L, name).restype = i32
+    return L
+
+
+lib = _load()
+
+
+class SparstarError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__("%s: %s (%d)" % (where, lib.sparstar_strerror(code).decode(), code))
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise SparstarError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    return t
+
+
+def nblocks(L: int) -> int:
+    return (L + BLOCK - 1) // BLOCK
+
+
+def default_tau(D: int) -> float:
+    return float(torch.tensor(1.0 / math.sqrt(D), dtype=torch.float32))
+
+
+def sparstar_forced_blocks(text_len: int, image_ref_len: int) -> int:
+    return lib.sparstar_forced_blocks(text_len, image_ref_len)
+
+
+def sparstar_select_count(nKB: int, n_forced_blocks: int, density: float) -> int:
+    return lib.sparstar_select_count(nKB, n_forced_blocks, density)
+
+
+def sparstar_block_pool(x: torch.Tensor, xbar: torch.Tensor = None, stream=None) -> torch.Tensor:
+    _dev(x, "x")
+    B, H, L, D = x.shape
+    if xbar is None:
+        xbar = torch.empty(B, H, nblocks(L), D, device=x.device, dtype=torch.float32)
+    _dev(xbar, "xbar", torch.float32)
+    _check(lib.sparstar_block_pool(_ptr(x), _DTYPE.get(x.dtype, -1), B, H, L, D, _ptr(xbar),
+                                   _stream(stream)), "sparstar_block_pool")
+    return xbar
+
+
+def sparstar_block_score(qbar: torch.Tensor, kbar: torch.Tensor, tau: float = None,
+                         S: torch.Tensor = None, stream=None) -> torch.Tensor:
+    _dev(qbar, "qbar", torch.float32)
+    _dev(kbar, "kbar", torch.float32)
+    B, H, nQB, D = qbar.shape
+    nKB = kbar.shape[2]
+    if tau is None:
+        tau = default_tau(D)
+    if S is None:
+        S = torch.empty(B, H, nQB, nKB, device=qbar.device, dtype=torch.float32)
+    _dev(S, "S", torch.float32)
+    _check(lib.sparstar_block_score(_ptr(qbar), _ptr(kbar), B, H, nQB, nKB, D, tau, _ptr(S),
+                                    _stream(stream)), "sparstar_block_score")
+    return S
+
+
+def sparstar_select(S: torch.Tensor, n_forced_blocks: int, density: float, max_sel: int = None,
+                    kv_idx: torch.Tensor = None, kv_cnt: torch.Tensor = None, stream=None):
+    _dev(S, "S", torch.float32)
+    B, H, nQB, nKB = S.shape
+    if max_sel is None:
+        max_sel = kv_idx.shape[-1] if kv_idx is not None else \
+            sparstar_select_count(nKB, n_forced_blocks, density)
+        if max_sel < 0:
+            raise SparstarError(EINVAL, "sparstar_select")
+    if kv_idx is None:
+        kv_idx = torch.empty(B, H, nQB, max_sel, device=S.device, dtype=torch.int32)
+    if kv_cnt is None:
+        kv_cnt = torch.empty(B, H, nQB, device=S.device, dtype=torch.int32)
+    _dev(kv_idx, "kv_idx", torch.int32)
+    _dev(kv_cnt, "kv_cnt", torch.int32)
+    _check(lib.sparstar_select(_ptr(S), B, H, nQB, nKB, n_forced_blocks, density, _ptr(kv_idx),
+                               _ptr(kv_cnt), max_sel, _stream(stream)), "sparstar_select")
+    return kv_idx, kv_cnt
+
+
+def sparstar_attn_fwd(q, k, v, kv_idx, kv_cnt, tau: float = None, out=None, lse=None,
+                      status=None, want_lse: bool = True, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    _dev(kv_idx, "kv_idx", torch.int32)
+    _dev(kv_cnt, "kv_cnt", torch.int32)
+    B, H, Lq, D = q.shape
+    Lk = k.shape[2]
+    if tau is None:
+        tau = default_tau(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, Lq, device=q.device, dtype=torch.float32)
+    _check(lib.sparstar_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _DTYPE.get(q.dtype, -1), B, H, Lq,
+                                 Lk, D, tau, _ptr(kv_idx), _ptr(kv_cnt), kv_idx.shape[-1],
+                                 _ptr(out), _ptr(lse), _ptr(status), _stream(stream)),
+           "sparstar_attn_fwd")
+    return out, lse
+
+
+class Workspace:
+    """Caller-owned device buffers for one scale of ``sparstar_forward``."""
+
+    def __init__(self, B, H, D, text_len, image_ref_len, ref_len, cur_len, density, device):
+        Lk = text_len + image_ref_len + ref_len + cur_len
+        self.nQB, self.nKB = nblocks(cur_len), nblocks(Lk)
+        self.n_forced = sparstar_forced_blocks(text_len, image_ref_len)
+        self.max_sel = sparstar_select_count(self.nKB, self.n_forced, density)
+        if self.max_sel < 0:
+            raise SparstarError(EINVAL, "Workspace")
+        f32, i32 = torch.float32, torch.int32
+        self.qbar = torch.empty(B, H, self.nQB, D, device=device, dtype=f32)
+        self.kbar = torch.empty(B, H, self.nKB, D, device=device, dtype=f32)
+        self.S = torch.empty(B, H, self.nQB, self.nKB, device=device, dtype=f32)
+        self.kv_idx = torch.empty(B, H, self.nQB, self.max_sel, device=device, dtype=i32)
+        self.kv_cnt = torch.empty(B, H, self.nQB, device=device, dtype=i32)
+
+
+def sparstar_forward(q, k, v, text_len, image_ref_len, ref_len, cur_len, density,
+                     workspace: Workspace = None, out=None, lse=None, status=None,
+                     want_lse: bool = True, stream=None):
+    """All four steps for one scale on one stream; returns (out, lse, workspace)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, H, Lq, D = q.shape
+    ws = workspace or Workspace(B, H, D, text_len, image_ref_len, ref_len, cur_len, density,
+                                q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, Lq, device=q.device, dtype=torch.float32)
+    _check(lib.sparstar_forward(_ptr(q), _ptr(k), _ptr(v), _DTYPE.get(q.dtype, -1), B, H, D,
+                                text_len, image_ref_len, ref_len, cur_len, density, _ptr(ws.qbar),
+                                _ptr(ws.kbar), _ptr(ws.S), _ptr(ws.kv_idx), _ptr(ws.kv_cnt),
+                                ws.max_sel, _ptr(out), _ptr(lse), _ptr(status), _stream(stream)),
+           "sparstar_forward")
+    return out, lse, ws

@@ -1,0 +1,187 @@
+/*
+ * sparstar.h — C ABI of libsparstar: SparSTAR's per-scale block-sparse
+ * attention forward on B200 (sm_100a).
+ *
+ * The operation (SparSTAR, arXiv 2608.10519; pith.science review of the
+ * paper, "What carries the argument"): at one expensive scale, per attention
+ * head,
+ *   1. average Q and K over contiguous 128-token blocks;
+ *   2. score every (query block i, key block j) pair as
+ *      S_ij = tau * qbar_i^T kbar_j, tau = D^-1/2 (the paper's Eq. 2), keep
+ *      the text blocks (and, for Clip 1, the image-pyramid reference blocks)
+ *      by force, and keep the top ceil(density * C) of the remaining C
+ *      reference and current-scale blocks, ranked jointly;
+ *   3. run a forward-only attention over the selected 128 x 128 tiles only,
+ *      described by a forward block list (per-row count + key-block index
+ *      list) without any reverse index.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are [B, H, L, D] row-major, D contiguous, with no padding.
+ *    Key order inside L_k: [text | image_ref | ref | cur]; queries are the
+ *    current-scale tokens.  Blocks are 128 tokens; the last block of a grid
+ *    may be partial and then holds L - 128 * (nblocks - 1) real tokens.
+ *  - Pointers passed to kernels are DEVICE pointers (cudaMalloc'd or
+ *    equivalent), owned by the caller; the library allocates no memory,
+ *    keeps no state between calls and never synchronises.  `stream` is a
+ *    cudaStream_t handle (NULL = the legacy default stream); every call is
+ *    asynchronous on it.
+ *  - dtype codes: SPARSTAR_BF16 = 0 (bfloat16 stored as 16-bit words),
+ *    SPARSTAR_F32 = 1.  Head dim D is 64 or 128.
+ *  - Return value: SPARSTAR_OK (0) or an error code below.  Argument errors
+ *    are detected on the host before anything is launched; SPARSTAR_ECUDA
+ *    reports a launch failure (cudaGetLastError after the launch).
+ *  - Device pointers to q, k, v, out and the pooled / score buffers must be
+ *    16-byte aligned (cudaMalloc gives 256).
+ *  - The library is built for sm_100a only; calls on another device return
+ *    SPARSTAR_ENODEV.
+ */
+#ifndef SPARSTAR_H
+#define SPARSTAR_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPARSTAR_BLOCK 128
+
+enum sparstar_dtype { SPARSTAR_BF16 = 0, SPARSTAR_F32 = 1 };
+
+enum sparstar_status {
+    SPARSTAR_OK = 0,
+    SPARSTAR_EINVAL = 1,  /* bad size, null pointer, misalignment, density outside (0,1] */
+    SPARSTAR_EDTYPE = 2,  /* unknown dtype code */
+    SPARSTAR_ECUDA = 3,   /* a CUDA runtime call or launch failed */
+    SPARSTAR_ESIZE = 4,   /* output list too small (max_sel < selected count) */
+    SPARSTAR_ENODEV = 5   /* no usable sm_100 device for this call */
+};
+
+/* Bits the attention kernels OR into *status (when status is non-NULL). */
+#define SPARSTAR_STATUS_BAD_INDEX 0x1 /* a kv_idx entry outside [0, nKB) was skipped */
+#define SPARSTAR_STATUS_TIMEOUT 0x2   /* a pipeline wait gave up; output is invalid */
+
+/*
+ * sparstar_block_pool — step 1, block mean pooling.
+ * Passage: "block-averaged query and key vectors over contiguous 128-token
+ * blocks in attention-kernel order" ([R-carry] above).
+ *   x     [B,H,L,D] of `dtype` (device)
+ *   xbar  [B,H,ceil(L/128),D] fp32 (device, written)
+ * xbar[b,h,blk,d] is the mean of the block's real tokens, summed in this
+ * fixed fp32 order: stripe r = 0..7 adds the tokens t = r, r+8, r+16, ...
+ * of the block in ascending t, starting from +0; the total is
+ * ((s0+s1)+(s2+s3))+((s4+s5)+(s6+s7)); the mean is one IEEE
+ * round-to-nearest division by the real token count n.
+ * Call once for Q (L = Lq) and once for K (L = Lk).
+ */
+int sparstar_block_pool(const void *x, int dtype, int64_t B, int64_t H, int64_t L,
+                        int64_t D, float *xbar, void *stream);
+
+/*
+ * sparstar_block_score — step 2a, the aggregated block score (Eq. 2).
+ * Passage: "S_ij = tau qbar_i^T kbar_j ... tau = D^-1/2" and "the dot
+ * product of block averages equals the average pairwise pre-softmax
+ * compatibility" ([R-carry]).
+ *   qbar [B,H,nQB,D] fp32, kbar [B,H,nKB,D] fp32 (device)
+ *   tau  fp32 scale, normally (float)(1/sqrt((double)D))
+ *   S    [B,H,nQB,nKB] fp32 (device, written)
+ * S = (acc) * tau, one IEEE multiply, where acc starts at +0 and takes
+ * acc = fma(qbar[d], kbar[d], acc) for d = 0..D-1 in ascending order.
+ * Every pair is scored, forced blocks included.  Results are bit-identical
+ * to any implementation of that order.
+ */
+int sparstar_block_score(const float *qbar, const float *kbar, int64_t B, int64_t H,
+                         int64_t nQB, int64_t nKB, int64_t D, float tau, float *S,
+                         void *stream);
+
+/*
+ * sparstar_forced_blocks — host only.  Number of leading key blocks that
+ * hold at least one text or Clip-1 image-reference token:
+ * ceil((text_len + image_ref_len) / 128).  Passage: text (and, for Clip 1,
+ * the final image-pyramid reference) "are always retained dense"
+ * ([R-carry]).  Returns -1 for negative lengths.
+ */
+int64_t sparstar_forced_blocks(int64_t text_len, int64_t image_ref_len);
+
+/*
+ * sparstar_select_count — host only.  Selected blocks per query block:
+ * n_forced_blocks + k with k = ceil(density * C), C = nKB - n_forced_blocks,
+ * computed in fp64 and clamped to [0, C].  Passage: the per-scale density
+ * schedule ([R-carry]).  Returns -1 when nKB <= 0, n_forced_blocks is
+ * outside [0, nKB] or density is outside (0, 1].
+ */
+int64_t sparstar_select_count(int64_t nKB, int64_t n_forced_blocks, double density);
+
+/*
+ * sparstar_select — step 2b, clip-aware block Top-K into a forward-only
+ * block list.  Passage: text / Clip-1 reference retained; "preceding-clip
+ * reference and current-scale blocks are jointly ranked under the density
+ * schedule"; FastFlex "writes only the forward mask fields and skips
+ * reverse-index construction" ([R-carry]).
+ *   S       [B,H,nQB,nKB] fp32 (device); must be finite
+ *   kv_idx  [B,H,nQB,max_sel] int32 (device, written): for every row,
+ *           0..nF-1, then the chosen candidates in ascending order, then -1
+ *           in the unused slots
+ *   kv_cnt  [B,H,nQB] int32 (device, written): sel = sparstar_select_count
+ * Candidates j in [nF, nKB) are ranked by S descending, equal scores
+ * (with -0 == +0) going to the lower j.  Returns SPARSTAR_ESIZE when
+ * max_sel < sel.
+ */
+int sparstar_select(const float *S, int64_t B, int64_t H, int64_t nQB, int64_t nKB,
+                    int64_t n_forced_blocks, double density, int32_t *kv_idx,
+                    int32_t *kv_cnt, int64_t max_sel, void *stream);
+
+/*
+ * sparstar_attn_fwd — step 3, forward attention over the listed tiles.
+ * Passage: SparSTAR "executes the selected blocks through a forward-only
+ * sparse path" (abstract); the chosen blocks run through a forward-only
+ * attention ([R-carry]).
+ *   q [B,H,Lq,D], k and v [B,H,Lk,D] of `dtype` (device)
+ *   tau      softmax scale (normally D^-1/2)
+ *   kv_idx   [B,H,ceil(Lq/128),max_sel] int32, kv_cnt [B,H,ceil(Lq/128)]
+ *            int32 (device): the block list of each query block.  Entries
+ *            past kv_cnt are ignored; an entry outside [0, ceil(Lk/128)) is
+ *            skipped and flagged in *status.
+ *   out      [B,H,Lq,D] of `dtype` (device, written)
+ *   lse      [B,H,Lq] fp32 natural-log sum-exp of the scaled scores over
+ *            the visible keys (device, written), or NULL
+ *   status   one int32 (device) that kernels OR SPARSTAR_STATUS_* bits into,
+ *            or NULL; the caller zeroes it
+ * For query row r of block i: out_r = sum_t softmax_t(tau q_r.k_t) v_t over
+ * the tokens t < Lk of the listed key blocks.  No causal mask.  A row whose
+ * list is empty gets out = 0 and lse = -inf.  bf16 with D = 128 runs on the
+ * tcgen05 tensor-core kernel (fp32 accumulation and softmax, P rounded to
+ * bf16 for the second product); fp32 inputs and D = 64 run on an fp32 SIMT
+ * kernel.
+ */
+int sparstar_attn_fwd(const void *q, const void *k, const void *v, int dtype, int64_t B,
+                      int64_t H, int64_t Lq, int64_t Lk, int64_t D, float tau,
+                      const int32_t *kv_idx, const int32_t *kv_cnt, int64_t max_sel,
+                      void *out, float *lse, int32_t *status, void *stream);
+
+/*
+ * sparstar_forward — the four steps in order on one stream, for one scale.
+ * Segments: text_len, image_ref_len (Clip 1 only, else 0), ref_len, cur_len;
+ * Lk = their sum, Lq = cur_len.  Workspace (device, caller-owned):
+ *   qbar [B,H,nQB,D] fp32, kbar [B,H,nKB,D] fp32, S [B,H,nQB,nKB] fp32,
+ *   kv_idx [B,H,nQB,max_sel] int32, kv_cnt [B,H,nQB] int32.
+ * tau = (float)(1/sqrt(D)).  Returns the first error of the chain.
+ */
+int sparstar_forward(const void *q, const void *k, const void *v, int dtype, int64_t B,
+                     int64_t H, int64_t D, int64_t text_len, int64_t image_ref_len,
+                     int64_t ref_len, int64_t cur_len, double density, float *qbar,
+                     float *kbar, float *S, int32_t *kv_idx, int32_t *kv_cnt,
+                     int64_t max_sel, void *out, float *lse, int32_t *status, void *stream);
+
+/* Message for a status code (static storage). */
+const char *sparstar_strerror(int code);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int sparstar_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSTAR_H */
