@@ -4,26 +4,35 @@
 // forward-only attention; the block list holds only forward fields).
 //
 // One CTA per (b, h, query block) in head-major order, so the CTAs that run
-// together share one head's K/V in L2.  Six warps, specialised:
-//   warps 0-3  softmax + epilogue: thread r owns query row r = TMEM lane r;
-//   warp 4     TMA producer: Q once, then K/V tiles in consumption order
+// together share one head's K/V in L2.  Ten warps, specialised:
+//   warps 0-7  softmax + epilogue.  Warp w serves TMEM lanes 32*(w%4)..+31
+//              (query rows) and half h = w/4 of each key tile (keys
+//              64h..64h+63), so every query row is owned by two threads and
+//              each SM sub-partition runs two softmax warps;
+//   warp 8     TMA producer: Q once, then K/V tiles in consumption order
 //              K0, K1, V0, K2, V1, ..., V(n-1) through a 6-stage ring;
-//   warp 5     TMEM allocation and the single MMA-issuing thread.
-// TMEM (512 columns): S double buffer at columns 0 and 128 (fp32 128 x 128),
-// O accumulator at column 256.  P_j (bf16) is written over the first 64
-// columns of S_j's buffer and feeds the second product straight from TMEM
-// (tcgen05.mma with A in tensor memory), so P never touches shared memory.
+//   warp 9     TMEM allocation and the single MMA-issuing thread.
+// TMEM (512 columns): S double buffer at columns 0 and 128 (fp32 128 x 128);
+// two O accumulators, O_0 at 256 and O_1 at 384, one per key half.  P of
+// half h (bf16, packed two per column) is written over columns 64h..64h+31
+// of the S buffer it came from (inside the columns the same thread read)
+// and feeds the second product straight from TMEM (tcgen05.mma with A in
+// tensor memory), so P never touches shared memory.
 //
 // Per tile j: S_j = Q K_j^T (8 MMAs of K = 16, A = Q and B = K both
 // K-major, 128-byte swizzle), the softmax turns S_j into P_j, then
-// O += P_j V_j (8 MMAs, A = P from TMEM, B = V MN-major).  The MMA thread
-// issues S_{j+1} before waiting for P_j, so the tensor core computes the
-// next scores while the softmax runs.
+// O_h += P_j,h V_j[64h..64h+63] for h = 0, 1 (4 MMAs each, A = P from
+// TMEM, B = V MN-major).  The MMA thread issues S_{j+1} before waiting for
+// P_j, so the tensor core computes the next scores while the softmax runs.
 //
-// Online softmax in the log2 domain: scores are scaled by tau * log2(e);
-// a row keeps a reference max m and only rescales O and l when the tile max
-// exceeds m by more than 8 (a factor 256), which keeps P below 256 and
-// makes the O rescale (a TMEM round trip) rare.
+// Each key half runs its own online softmax (running max m_h, sum l_h,
+// accumulator O_h), so the two threads of a row never synchronise inside
+// the loop; the halves are merged once in the epilogue:
+//   M = max(m_0, m_1), O = sum_h 2^(m_h - M) O_h / sum_h 2^(m_h - M) l_h.
+// Scores are kept in log2 units (scaled by tau * log2(e)); a half only
+// rescales O_h and l_h when its tile max exceeds m_h by more than 8 (a
+// factor 256), which keeps P below 256 and makes the O rescale (a TMEM
+// round trip) rare.
 //
 // Every wait is bounded (about two seconds of %globaltimer): on expiry the
 // CTA raises SPARSTAR_STATUS_TIMEOUT in *status, every role leaves its
@@ -43,11 +52,12 @@ constexpr int kHD = 128;                  // head dim
 constexpr int kStages = 6;                // K/V ring depth
 constexpr int kTileBytes = kBlock * kHD * 2;  // 32 KB: one Q, K or V tile
 constexpr int kPanelBytes = kTileBytes / 2;   // 16 KB: 128 rows x 64 columns
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4, kMmaWarp = 5;
+constexpr int kSoftmaxThreads = 256;  // warps 0-7
+constexpr int kThreads = kSoftmaxThreads + 64;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int b) { return (b & 1) ? 128u : 0u; }  // S buffers
-constexpr uint32_t kColO = 256;
+__host__ __device__ constexpr uint32_t col_o(int h) { return h ? 384u : 256u; }  // O_0, O_1
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
@@ -258,6 +268,13 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
     return *reinterpret_cast<uint32_t *>(&h);
@@ -314,7 +331,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             }
             for (int b = 0; b < 2; ++b) {
                 mbar_init(bar_s(b), 1);
-                mbar_init(bar_p(b), 128);
+                mbar_init(bar_p(b), kSoftmaxThreads);
                 mbar_init(bar_pv(b), 1);
             }
             mbar_init(bar_drain, 1);
@@ -397,11 +414,14 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     return false;
                 tc_fence_after();
                 const uint32_t sV = base + kOffStage + stage * kTileBytes;
+                // O_h += P_h V[64h .. 64h+63]; P_h sits at S columns 64h..64h+31.
 #pragma unroll
-                for (int kk = 0; kk < kBlock / 16; ++kk)
-                    mma_ts(tmem + kColO, tmem + col_s(jj & 1) + (uint32_t)(kk * 8),
-                           desc_mn_major(sV + kk * 16 * 128), kIdescPV,
-                           (jj > 0 || kk > 0) ? 1u : 0u);
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + col_o(h), tmem + col_s(jj & 1) + 64u * h + 8u * kk,
+                               desc_mn_major(sV + (4 * h + kk) * 16 * 128), kIdescPV,
+                               (jj > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar_empty(stage));
                 mma_commit(bar_pv(jj & 1));
                 ++e;
@@ -435,9 +455,12 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
         __syncwarp();
     } else {
-        // ------------------------------------------- softmax + epilogue (128 thr)
-        const int row = warp * 32 + lane;  // TMEM lane == tile row
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // ------------------------------------------ softmax + epilogue (256 thr)
+        const int quarter = warp & 3;      // TMEM lane quarter
+        const int half = warp >> 2;        // key half of every tile
+        const int row = quarter * 32 + lane;  // TMEM lane == tile row
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        const uint32_t colO = col_o(half);
         const float sc = tau * 1.4426950408889634f;  // scores in log2 units
         float m_ref = -INFINITY, l = 0.0f;
         bool ok = true;
@@ -449,34 +472,33 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 break;
             }
             tc_fence_after();
-            float s[kBlock];
+            const uint32_t colS = col_s(j & 1) + 64u * half;
+            float s[64];
             {
-                uint32_t r[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + col_s(j & 1) + 32 * c, r[c]);
+                uint32_t r[2][32];
+                tmem_ld32(tmem + lane_base + colS, r[0]);
+                tmem_ld32(tmem + lane_base + colS + 32, r[1]);
                 tmem_wait_ld();
+                reg_fence(r[0]);
+                reg_fence(r[1]);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) reg_fence(r[c]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int u = 0; u < 32; ++u) s[32 * c + u] = __uint_as_float(r[c][u]);
             }
-            const int valid = Lk - kb * kBlock;  // keys of this tile that exist
-            if (valid < kBlock) {
+            const int valid = Lk - kb * kBlock - 64 * half;  // keys of this half that exist
+            if (valid < 64) {
 #pragma unroll
-                for (int c = 0; c < kBlock; ++c)
+                for (int c = 0; c < 64; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+            float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int c = 4; c < kBlock; c += 4) {
-                mx0 = fmaxf(mx0, s[c]);
-                mx1 = fmaxf(mx1, s[c + 1]);
-                mx2 = fmaxf(mx2, s[c + 2]);
-                mx3 = fmaxf(mx3, s[c + 3]);
+            for (int c = 4; c < 64; c += 8) {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) mx[t] = max3f(mx[t], s[c + t], s[c + 4 + t]);
             }
-            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc;
+            const float m_tile = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
             const float m_new = fmaxf(m_ref, m_tile);
             if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
                 if (j > 0) {
@@ -486,87 +508,114 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         break;
                     }
                     tc_fence_after();
-                    const float f = ex2(m_ref - m_new);
+                    const float f = m_new > -INFINITY ? ex2(m_ref - m_new) : 1.0f;  // 0 if no key seen yet
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t r[32];
-                        tmem_ld32(tmem + lane_base + kColO + 32 * c, r);
+                        tmem_ld32(tmem + lane_base + colO + 32 * c, r);
                         tmem_wait_ld();
                         reg_fence(r);
 #pragma unroll
                         for (int u = 0; u < 32; ++u)
                             r[u] = __float_as_uint(__uint_as_float(r[u]) * f);
-                        tmem_st32(tmem + lane_base + kColO + 32 * c, r);
+                        tmem_st32(tmem + lane_base + colO + 32 * c, r);
                     }
                     tmem_wait_st();
                 }
-                l *= ex2(m_ref - m_new);  // l = 0 on the first tile
-                m_ref = m_new;
-            }
-            float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int u = 0; u < 32; u += 2) {
-                    const int c = 64 * h + 2 * u;
-                    const float p0 = ex2(fmaf(s[c], sc, -m_ref));
-                    const float p1 = ex2(fmaf(s[c + 1], sc, -m_ref));
-                    const float p2 = ex2(fmaf(s[c + 2], sc, -m_ref));
-                    const float p3 = ex2(fmaf(s[c + 3], sc, -m_ref));
-                    ls0 += p0;
-                    ls1 += p1;
-                    ls2 += p2;
-                    ls3 += p3;
-                    pk[u] = pack_bf16(p0, p1);
-                    pk[u + 1] = pack_bf16(p2, p3);
+                if (m_new > -INFINITY) {  // a half with no key yet keeps l = 0
+                    l *= ex2(m_ref - m_new);
+                    m_ref = m_new;
                 }
-                tmem_st32(tmem + lane_base + col_s(j & 1) + 32 * h, pk);
             }
-            l += (ls0 + ls1) + (ls2 + ls3);
+            // m_ref = -inf only while every key of this half so far was masked:
+            // then every p is 0 (a finite offset keeps -inf * sc + offset = -inf).
+            const float neg_m = m_ref > -INFINITY ? -m_ref : 0.0f;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[32];
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) {
+                const int c = 2 * u;
+                const float p0 = ex2(fmaf(s[c], sc, neg_m));
+                const float p1 = ex2(fmaf(s[c + 1], sc, neg_m));
+                const float p2 = ex2(fmaf(s[c + 2], sc, neg_m));
+                const float p3 = ex2(fmaf(s[c + 3], sc, neg_m));
+                ls[0] += p0;
+                ls[1] += p1;
+                ls[2] += p2;
+                ls[3] += p3;
+                pk[u] = pack_bf16(p0, p1);
+                pk[u + 1] = pack_bf16(p2, p3);
+            }
+            tmem_st32(tmem + lane_base + colS, pk);
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p(j & 1));
         }
-        // ---- epilogue: O / l -> bf16, LSE
+
+        // ---- epilogue: merge the two halves, O / l -> bf16, LSE
+        const bool have = n > 0 && ok &&
+                          wait_warp(bar_pv((n - 1) & 1), (uint32_t)((n - 1) >> 1) & 1u, abort_flag,
+                                    status);
+        // Exchange (m, l) with the partner thread of the other half.  Every
+        // MMA has completed once the last O update has (or the CTA is
+        // aborting), so the Q tile's shared memory is free for this.
+        float *xm = reinterpret_cast<float *>(smem + kOffQ);  // [2][128]
+        float *xl = xm + 2 * kBlock;                           // [2][128]
+        xm[half * kBlock + row] = m_ref;
+        xl[half * kBlock + row] = l;
+        asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+        const float m_o = xm[(half ^ 1) * kBlock + row];
+        const float l_o = xl[(half ^ 1) * kBlock + row];
+        const float M = fmaxf(m_ref, m_o);
+        const float a_self = m_ref > -INFINITY ? ex2(m_ref - M) : 0.0f;
+        const float a_oth = m_o > -INFINITY ? ex2(m_o - M) : 0.0f;
+        const float L = l * a_self + l_o * a_oth;
+        const float a0 = half == 0 ? a_self : a_oth;  // weight of O_0
+        const float a1 = half == 0 ? a_oth : a_self;  // weight of O_1
+
         const int64_t grow = (int64_t)qb * kBlock + row;
         const bool store = grow < Lq;
-        __nv_bfloat16 *orow = out + ((int64_t)bh * Lq + grow) * kHD;
+        __nv_bfloat16 *orow = out + ((int64_t)bh * Lq + grow) * kHD + 64 * half;
         if (n == 0) {
             if (store) {
                 uint4 *o4 = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-                for (int c = 0; c < kHD / 8; ++c) o4[c] = make_uint4(0, 0, 0, 0);
-                if (lse) lse[(int64_t)bh * Lq + grow] = -INFINITY;
+                for (int c = 0; c < 8; ++c) o4[c] = make_uint4(0, 0, 0, 0);
+                if (lse && half == 0) lse[(int64_t)bh * Lq + grow] = -INFINITY;
             }
-        } else if (ok && wait_warp(bar_pv((n - 1) & 1), (uint32_t)((n - 1) >> 1) & 1u, abort_flag,
-                                   status)) {
+        } else if (have) {
             tc_fence_after();
-            const float inv = 1.0f / l;
+            const float inv = 1.0f / L;
+            const float w0 = a0 * inv, w1 = a1 * inv;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + kColO + 32 * c, r);
+            for (int c = 0; c < 2; ++c) {  // output columns 64*half + 32c .. +31
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_base + col_o(0) + 64 * half + 32 * c, r0);
+                tmem_ld32(tmem + lane_base + col_o(1) + 64 * half + 32 * c, r1);
                 tmem_wait_ld();
-                reg_fence(r);
+                reg_fence(r0);
+                reg_fence(r1);
                 if (store) {
                     uint4 *o4 = reinterpret_cast<uint4 *>(orow + 32 * c);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(r[8 * u + 0]) * inv,
-                                        __uint_as_float(r[8 * u + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(r[8 * u + 2]) * inv,
-                                        __uint_as_float(r[8 * u + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(r[8 * u + 4]) * inv,
-                                        __uint_as_float(r[8 * u + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(r[8 * u + 6]) * inv,
-                                        __uint_as_float(r[8 * u + 7]) * inv);
-                        o4[u] = w;
+                        float f[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t)
+                            f[t] = __uint_as_float(r0[8 * u + t]) * w0 +
+                                   __uint_as_float(r1[8 * u + t]) * w1;
+                        uint4 wv;
+                        wv.x = pack_bf16(f[0], f[1]);
+                        wv.y = pack_bf16(f[2], f[3]);
+                        wv.z = pack_bf16(f[4], f[5]);
+                        wv.w = pack_bf16(f[6], f[7]);
+                        o4[u] = wv;
                     }
                 }
             }
-            if (store && lse) lse[(int64_t)bh * Lq + grow] = (m_ref + log2f(l)) * 0.6931471805599453f;
+            if (store && lse && half == 0)
+                lse[(int64_t)bh * Lq + grow] = (M + log2f(L)) * 0.6931471805599453f;
         }
     }
 
