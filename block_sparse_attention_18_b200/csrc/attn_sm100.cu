@@ -268,6 +268,17 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// True in exactly one lane of the (fully active) warp.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .b32 r;\n\t.reg .pred p;\n\t"
+        "elect.sync r|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Three-input maximum (one instruction on sm_100).
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
@@ -401,57 +412,73 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t sQ = base + kOffQ;
-            int e = 0;
-            bool ok = n > 0 && wait1(bar_q, 0, abort_flag, status);
-            tc_fence_after();
-            auto issue_pv = [&](int jj) -> bool {
-                if (!wait1(bar_p(jj & 1), (uint32_t)(jj >> 1) & 1u, abort_flag, status))
-                    return false;
+        // The whole warp runs the control flow, so descriptors and TMEM
+        // addresses stay warp-uniform (no per-MMA register moves); one
+        // elected lane issues.  Descriptors are built once per operand and
+        // advanced by compile-time offsets.
+        const uint64_t dQ = desc_k_major(base + kOffQ);
+        int e = 0;
+        bool ok = n > 0 && wait_warp(bar_q, 0, abort_flag, status);
+        tc_fence_after();
+        for (int j = 0; j <= n && ok; ++j) {
+            if (j < n) {
+                // S_j = Q K_j^T
                 const int stage = e % kStages;
-                if (!wait1(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status))
-                    return false;
-                tc_fence_after();
-                const uint32_t sV = base + kOffStage + stage * kTileBytes;
-                // O_h += P_h V[64h .. 64h+63]; P_h sits at S columns 64h..64h+31.
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + col_o(h), tmem + col_s(jj & 1) + 64u * h + 8u * kk,
-                               desc_mn_major(sV + (4 * h + kk) * 16 * 128), kIdescPV,
-                               (jj > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar_empty(stage));
-                mma_commit(bar_pv(jj & 1));
-                ++e;
-                return true;
-            };
-            for (int j = 0; j < n && ok; ++j) {
-                const int stage = e % kStages;
-                if (!wait1(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
+                if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sK = base + kOffStage + stage * kTileBytes;
+                const uint64_t dK = desc_k_major(base + kOffStage + stage * kTileBytes);
+                const uint32_t dS = tmem + col_s(j & 1);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < kHD / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * kPanelBytes + (kk & 3) * 32);
-                    mma_ss(tmem + col_s(j & 1), desc_k_major(sQ + off), desc_k_major(sK + off),
-                           kIdescQK, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kHD / 16; ++kk) {
+                        const uint64_t off = (uint64_t)(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
+                        mma_ss(dS, dQ + off, dK + off, kIdescQK, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar_empty(stage));
+                    mma_commit(bar_s(j & 1));
                 }
-                mma_commit(bar_empty(stage));
-                mma_commit(bar_s(j & 1));
+                __syncwarp();
                 ++e;
-                if (j > 0 && !issue_pv(j - 1)) ok = false;
             }
-            if (ok && n > 0) issue_pv(n - 1);
-            // Drain: every MMA issued so far completes before TMEM is freed.
-            if (e > 0) {
-                mma_commit(bar_drain);
-                drain_wait(bar_drain, 0);
+            if (j > 0) {
+                // O_h += P_{j-1},h V_{j-1}[64h .. 64h+63]
+                const int jj = j - 1;
+                if (!wait_warp(bar_p(jj & 1), (uint32_t)(jj >> 1) & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                const int stage = e % kStages;
+                if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t dV = desc_mn_major(base + kOffStage + stage * kTileBytes);
+                const uint32_t aP = tmem + col_s(jj & 1);
+                const uint32_t first = jj > 0 ? 1u : 0u;
+                if (elect_one()) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ts(tmem + col_o(h), aP + 64u * h + 8u * kk,
+                                   dV + (uint64_t)(((4 * h + kk) * 16 * 128) >> 4), kIdescPV,
+                                   kk > 0 ? 1u : first);
+                    mma_commit(bar_empty(stage));
+                    mma_commit(bar_pv(jj & 1));
+                }
+                __syncwarp();
+                ++e;
             }
+        }
+        // Drain: every MMA issued so far completes before TMEM is freed.
+        if (e > 0) {
+            if (elect_one()) mma_commit(bar_drain);
+            __syncwarp();
+            if (lane == 0) drain_wait(bar_drain, 0);
         }
         __syncwarp();
     } else {
