@@ -121,10 +121,10 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Single-thread bounded wait.  False on timeout (flag raised) or when
-// another role already raised the abort flag.
-__device__ __noinline__ bool wait1(uint32_t bar, uint32_t parity, volatile int32_t *abort_flag,
-                                   int32_t *status) {
-    if (mbar_test(bar, parity)) return true;
+// another role already raised the abort flag.  The polling loop is out of
+// line; the common case (phase already complete) costs one try_wait.
+__device__ __noinline__ bool wait1_slow(uint32_t bar, uint32_t parity,
+                                        volatile int32_t *abort_flag, int32_t *status) {
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_test(bar, parity)) return true;
@@ -139,6 +139,11 @@ __device__ __noinline__ bool wait1(uint32_t bar, uint32_t parity, volatile int32
     }
 }
 
+__device__ __forceinline__ bool wait1(uint32_t bar, uint32_t parity, volatile int32_t *abort_flag,
+                                      int32_t *status) {
+    return mbar_test(bar, parity) || wait1_slow(bar, parity, abort_flag, status);
+}
+
 // Bounded wait that ignores the abort flag: used on the way out, for work
 // already issued (copies in flight, MMAs to drain).
 __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity) {
@@ -150,9 +155,9 @@ __device__ __noinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 
 // Warp-uniform bounded wait for warp-collective roles: the warp leaves
 // together, so the .sync.aligned tcgen05 instructions after it stay
-// converged.
-__device__ __noinline__ bool wait_warp(uint32_t bar, uint32_t parity,
-                                       volatile int32_t *abort_flag, int32_t *status) {
+// converged.  Fast path inline (one try_wait per lane); polling out of line.
+__device__ __noinline__ bool wait_warp_slow(uint32_t bar, uint32_t parity,
+                                            volatile int32_t *abort_flag, int32_t *status) {
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 0;; ++it) {
         const bool ok = mbar_test(bar, parity);
@@ -171,6 +176,11 @@ __device__ __noinline__ bool wait_warp(uint32_t bar, uint32_t parity,
             if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
         }
     }
+}
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity,
+                                          volatile int32_t *abort_flag, int32_t *status) {
+    if (__all_sync(0xffffffffu, mbar_test(bar, parity))) return true;
+    return wait_warp_slow(bar, parity, abort_flag, status);
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
@@ -419,7 +429,6 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const uint64_t dQ = desc_k_major(base + kOffQ);
         int e = 0;
         bool ok = n > 0 && wait_warp(bar_q, 0, abort_flag, status);
-        tc_fence_after();
         for (int j = 0; j <= n && ok; ++j) {
             if (j < n) {
                 // S_j = Q K_j^T
@@ -428,7 +437,6 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     ok = false;
                     break;
                 }
-                tc_fence_after();
                 const uint64_t dK = desc_k_major(base + kOffStage + stage * kTileBytes);
                 const uint32_t dS = tmem + col_s(j & 1);
                 if (elect_one()) {
@@ -450,12 +458,12 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     ok = false;
                     break;
                 }
+                tc_fence_after();  // orders the softmax's tcgen05.st of P before the MMA
                 const int stage = e % kStages;
                 if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
                 const uint64_t dV = desc_mn_major(base + kOffStage + stage * kTileBytes);
                 const uint32_t aP = tmem + col_s(jj & 1);
                 const uint32_t first = jj > 0 ? 1u : 0u;
