@@ -4,14 +4,19 @@
 // forward-only attention; the block list holds only forward fields).
 //
 // One CTA per (b, h, query block) in head-major order, so the CTAs that run
-// together share one head's K/V in L2.  Ten warps, specialised:
+// together share one head's K/V in L2.  Eleven warps, specialised:
 //   warps 0-7  softmax + epilogue.  Warp w serves TMEM lanes 32*(w%4)..+31
 //              (query rows) and half h = w/4 of each key tile (keys
 //              64h..64h+63), so every query row is owned by two threads and
 //              each SM sub-partition runs two softmax warps;
 //   warp 8     TMA producer: Q once, then K/V tiles in consumption order
 //              K0, K1, V0, K2, V1, ..., V(n-1) through a 6-stage ring;
-//   warp 9     TMEM allocation and the single MMA-issuing thread.
+//   warp 9     TMEM allocation and the S = Q K^T MMAs;
+//   warp 10    the O += P V MMAs.
+// Two MMA warps, so each pays one wait/issue round per tile and the two
+// streams run side by side; the only cross-warp hazard (S_{j+2} written
+// over the buffer P_j is read from) is closed by the QK warp waiting for
+// the PV MMAs of tile j to complete.
 // TMEM (512 columns): S double buffer at columns 0 and 128 (fp32 128 x 128);
 // two O accumulators, O_0 at 256 and O_1 at 384, one per key half.  P of
 // half h (bf16, packed two per column) is written over columns 64h..64h+31
@@ -53,8 +58,8 @@ constexpr int kStages = 6;                // K/V ring depth
 constexpr int kTileBytes = kBlock * kHD * 2;  // 32 KB: one Q, K or V tile
 constexpr int kPanelBytes = kTileBytes / 2;   // 16 KB: 128 rows x 64 columns
 constexpr int kSoftmaxThreads = 256;  // warps 0-7
-constexpr int kThreads = kSoftmaxThreads + 64;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = kSoftmaxThreads + 96;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kPvWarp = 10;
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int b) { return (b & 1) ? 128u : 0u; }  // S buffers
 __host__ __device__ constexpr uint32_t col_o(int h) { return h ? 384u : 256u; }  // O_0, O_1
@@ -355,7 +360,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 mbar_init(bar_p(b), kSoftmaxThreads);
                 mbar_init(bar_pv(b), 1);
             }
-            mbar_init(bar_drain, 1);
+            mbar_init(bar_drain, 2);  // one commit from each MMA warp
             bars->abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)));
@@ -421,71 +426,81 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 drain_wait(bar_full(e % kStages), (uint32_t)(e / kStages) & 1u);
         }
     } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------- MMA issuer
+        // -------------------------------------------- S = Q K^T MMA issuer
         // The whole warp runs the control flow, so descriptors and TMEM
-        // addresses stay warp-uniform (no per-MMA register moves); one
-        // elected lane issues.  Descriptors are built once per operand and
-        // advanced by compile-time offsets.
+        // addresses stay warp-uniform; one elected lane issues.  Descriptors
+        // are built once per operand and advanced by compile-time offsets.
         const uint64_t dQ = desc_k_major(base + kOffQ);
-        int e = 0;
         bool ok = n > 0 && wait_warp(bar_q, 0, abort_flag, status);
-        for (int j = 0; j <= n && ok; ++j) {
-            if (j < n) {
-                // S_j = Q K_j^T
-                const int stage = e % kStages;
-                if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
-                    ok = false;
-                    break;
-                }
-                const uint64_t dK = desc_k_major(base + kOffStage + stage * kTileBytes);
-                const uint32_t dS = tmem + col_s(j & 1);
-                if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < kHD / 16; ++kk) {
-                        const uint64_t off = (uint64_t)(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
-                        mma_ss(dS, dQ + off, dK + off, kIdescQK, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar_empty(stage));
-                    mma_commit(bar_s(j & 1));
-                }
-                __syncwarp();
-                ++e;
+        for (int j = 0; j < n && ok; ++j) {
+            const int e = j == 0 ? 0 : 2 * j - 1;  // ring slot of K_j
+            const int stage = e % kStages;
+            if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
+                ok = false;
+                break;
             }
-            if (j > 0) {
-                // O_h += P_{j-1},h V_{j-1}[64h .. 64h+63]
-                const int jj = j - 1;
-                if (!wait_warp(bar_p(jj & 1), (uint32_t)(jj >> 1) & 1u, abort_flag, status)) {
+            if (j >= 2) {
+                // S buffer j&1 still holds P_{j-2} until its PV MMAs complete.
+                if (!wait_warp(bar_pv(j & 1), (uint32_t)((j - 2) >> 1) & 1u, abort_flag, status)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();  // orders the softmax's tcgen05.st of P before the MMA
-                const int stage = e % kStages;
-                if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
-                    ok = false;
-                    break;
-                }
-                const uint64_t dV = desc_mn_major(base + kOffStage + stage * kTileBytes);
-                const uint32_t aP = tmem + col_s(jj & 1);
-                const uint32_t first = jj > 0 ? 1u : 0u;
-                if (elect_one()) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(tmem + col_o(h), aP + 64u * h + 8u * kk,
-                                   dV + (uint64_t)(((4 * h + kk) * 16 * 128) >> 4), kIdescPV,
-                                   kk > 0 ? 1u : first);
-                    mma_commit(bar_empty(stage));
-                    mma_commit(bar_pv(jj & 1));
-                }
-                __syncwarp();
-                ++e;
+                tc_fence_after();
             }
+            const uint64_t dK = desc_k_major(base + kOffStage + stage * kTileBytes);
+            const uint32_t dS = tmem + col_s(j & 1);
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < kHD / 16; ++kk) {
+                    const uint64_t off = (uint64_t)(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
+                    mma_ss(dS, dQ + off, dK + off, kIdescQK, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar_empty(stage));
+                mma_commit(bar_s(j & 1));
+            }
+            __syncwarp();
         }
-        // Drain: every MMA issued so far completes before TMEM is freed.
-        if (e > 0) {
+        // Drain: every MMA this warp issued completes before TMEM is freed.
+        if (n > 0) {
             if (elect_one()) mma_commit(bar_drain);
             __syncwarp();
+        }
+    } else if (warp == kPvWarp) {
+        // ---------------------------------------------- O += P V MMA issuer
+        bool ok = n > 0;
+        for (int jj = 0; jj < n && ok; ++jj) {
+            if (!wait_warp(bar_p(jj & 1), (uint32_t)(jj >> 1) & 1u, abort_flag, status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();  // orders the softmax's tcgen05.st of P before the MMA
+            const int e = jj == n - 1 ? 2 * n - 1 : 2 * jj + 2;  // ring slot of V_jj
+            const int stage = e % kStages;
+            if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
+                ok = false;
+                break;
+            }
+            const uint64_t dV = desc_mn_major(base + kOffStage + stage * kTileBytes);
+            const uint32_t aP = tmem + col_s(jj & 1);
+            const uint32_t first = jj > 0 ? 1u : 0u;
+            if (elect_one()) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + col_o(h), aP + 64u * h + 8u * kk,
+                               dV + (uint64_t)(((4 * h + kk) * 16 * 128) >> 4), kIdescPV,
+                               kk > 0 ? 1u : first);
+                mma_commit(bar_empty(stage));
+                mma_commit(bar_pv(jj & 1));
+            }
+            __syncwarp();
+        }
+        if (n > 0) {
+            if (elect_one()) mma_commit(bar_drain);
+            __syncwarp();
+            // Both MMA warps have committed to the drain barrier; its phase
+            // completes once every MMA of the CTA has.
             if (lane == 0) drain_wait(bar_drain, 0);
         }
         __syncwarp();
