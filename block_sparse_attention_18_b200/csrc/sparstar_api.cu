@@ -55,7 +55,9 @@ SPARSTAR_API const char *sparstar_strerror(int code) {
     case SPARSTAR_EINVAL: return "invalid argument (size, null pointer, alignment or density)";
     case SPARSTAR_EDTYPE: return "unsupported dtype code";
     case SPARSTAR_ECUDA: return "CUDA runtime error";
-    case SPARSTAR_ESIZE: return "block list capacity max_sel below the selected count";
+    case SPARSTAR_ESIZE:
+        return "buffer too small: max_sel below the selected count, or the intermediates "
+               "exceed the static arena (SPARSTAR_STATIC_ARENA_BYTES)";
     case SPARSTAR_ENODEV: return "no sm_100 device available for this call";
     default: return "unknown status";
     }

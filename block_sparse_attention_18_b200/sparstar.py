@@ -41,6 +41,9 @@ def _load():
                                     vp, vp, vp, vp]
     L.sparstar_forward.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, f64, vp,
                                    vp, vp, vp, vp, i64, vp, vp, vp, vp]
+    L.sparstar_forward_static.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, f64,
+                                          vp, vp, vp, vp]
+    L.sparstar_forward_static.restype = i32
     L.sparstar_strerror.argtypes = [i32]
     L.sparstar_strerror.restype = ctypes.c_char_p
     L.sparstar_version.restype = i32
@@ -205,3 +208,23 @@ def sparstar_forward(q, k, v, text_len, image_ref_len, ref_len, cur_len, density
                                 ws.max_sel, _ptr(out), _ptr(lse), _ptr(status), _stream(stream)),
            "sparstar_forward")
     return out, lse, ws
+
+
+def sparstar_forward_static(q, k, v, text_len, image_ref_len, ref_len, cur_len, density,
+                            out=None, lse=None, status=None, want_lse: bool = True, stream=None):
+    """The four steps for one scale with the intermediates in the library's
+    own device arena (no workspace); returns (out, lse).  For callers that
+    cannot allocate device memory; calls that overlap on the GPU race on the
+    shared arena."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, H, Lq, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, Lq, device=q.device, dtype=torch.float32)
+    _check(lib.sparstar_forward_static(_ptr(q), _ptr(k), _ptr(v), _DTYPE.get(q.dtype, -1), B, H,
+                                       D, text_len, image_ref_len, ref_len, cur_len, density,
+                                       _ptr(out), _ptr(lse), _ptr(status), _stream(stream)),
+           "sparstar_forward_static")
+    return out, lse

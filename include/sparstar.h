@@ -23,7 +23,8 @@
  *    may be partial and then holds L - 128 * (nblocks - 1) real tokens.
  *  - Pointers passed to kernels are DEVICE pointers (cudaMalloc'd or
  *    equivalent), owned by the caller; the library allocates no memory,
- *    keeps no state between calls and never synchronises.  `stream` is a
+ *    keeps no state between calls and never synchronises (the one
+ *    exception, sparstar_forward_static, is described at its declaration).  `stream` is a
  *    cudaStream_t handle (NULL = the legacy default stream); every call is
  *    asynchronous on it.
  *  - dtype codes: SPARSTAR_BF16 = 0 (bfloat16 stored as 16-bit words),
@@ -39,6 +40,7 @@
 #ifndef SPARSTAR_H
 #define SPARSTAR_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -54,7 +56,7 @@ enum sparstar_status {
     SPARSTAR_EINVAL = 1,  /* bad size, null pointer, misalignment, density outside (0,1] */
     SPARSTAR_EDTYPE = 2,  /* unknown dtype code */
     SPARSTAR_ECUDA = 3,   /* a CUDA runtime call or launch failed */
-    SPARSTAR_ESIZE = 4,   /* output list too small (max_sel < selected count) */
+    SPARSTAR_ESIZE = 4,   /* max_sel < selected count, or a call too big for the static arena */
     SPARSTAR_ENODEV = 5   /* no usable sm_100 device for this call */
 };
 
@@ -173,6 +175,38 @@ int sparstar_forward(const void *q, const void *k, const void *v, int dtype, int
                      int64_t ref_len, int64_t cur_len, double density, float *qbar,
                      float *kbar, float *S, int32_t *kv_idx, int32_t *kv_cnt,
                      int64_t max_sel, void *out, float *lse, int32_t *status, void *stream);
+
+/*
+ * sparstar_forward_static — sparstar_forward for callers that cannot
+ * allocate device memory.  The paper has no counterpart: it is an
+ * allocation-free way into the same four steps.
+ *
+ * Some callers have no way to allocate device memory of their own: a host
+ * program that hands the library only its input and output buffers, or a
+ * plugin whose host forbids device allocations outside its own pool.  This
+ * entry point takes the same arguments as sparstar_forward minus the
+ * workspace and keeps the intermediates (block means, scores, block lists)
+ * in a fixed arena of SPARSTAR_STATIC_ARENA_BYTES that the library itself
+ * reserves on every GPU that loads it, for the life of the process.  It
+ * calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - Size limit: the intermediates of one call, 4 * B * H * (nQB * D +
+ *     nKB * D + nQB * nKB + nQB * sel + nQB) bytes plus alignment, must fit
+ *     in the arena (the 72,000-token scale with 16 heads needs about
+ *     59 MB); larger calls return SPARSTAR_ESIZE and launch nothing.
+ *   - The first call on each device looks the arena's address up
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls share the arena.  Calls whose GPU work overlaps (other
+ *     streams, other host threads) race on it; serialise them.
+ * The caller still owns q, k, v, out, lse and status.  Errors are those of
+ * sparstar_forward, plus SPARSTAR_ESIZE for a call that does not fit.
+ */
+#define SPARSTAR_STATIC_ARENA_BYTES ((size_t)64 << 20)
+
+int sparstar_forward_static(const void *q, const void *k, const void *v, int dtype, int64_t B,
+                            int64_t H, int64_t D, int64_t text_len, int64_t image_ref_len,
+                            int64_t ref_len, int64_t cur_len, double density, void *out,
+                            float *lse, int32_t *status, void *stream);
 
 /* Message for a status code (static storage). */
 const char *sparstar_strerror(int code);
