@@ -188,12 +188,26 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity,
     return wait_warp_slow(bar, parity, abort_flag, status);
 }
 
+// L2 eviction policies for TMA loads: Q tiles are read once per CTA
+// (evict first); K/V tiles, re-read by the other query blocks of the head,
+// keep the normal policy.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int c0, int c1, int c2) {
+                                            int c0, int c1, int c2, uint64_t policy) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
         : "memory");
 }
 
@@ -395,9 +409,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         // ------------------------------------------------------ TMA producer
         if (lane == 0 && n > 0) {
             const uint32_t sQ = base + kOffQ;
+            const uint64_t pol_q = policy_evict_first(), pol_kv = policy_evict_normal();
             mbar_expect_tx(bar_q, kTileBytes);
-            tma_load_3d(sQ, &tmQ, bar_q, 0, qb * kBlock, bh);
-            tma_load_3d(sQ + kPanelBytes, &tmQ, bar_q, 64, qb * kBlock, bh);
+            tma_load_3d(sQ, &tmQ, bar_q, 0, qb * kBlock, bh, pol_q);
+            tma_load_3d(sQ + kPanelBytes, &tmQ, bar_q, 64, qb * kBlock, bh, pol_q);
             int curK = 0, curV = 0;
             int issued = 0;
             bool ok = true;
@@ -414,8 +429,8 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 const uint32_t dst = base + kOffStage + stage * kTileBytes;
                 const CUtensorMap *map = is_v ? &tmV : &tmK;
                 mbar_expect_tx(bar_full(stage), kTileBytes);
-                tma_load_3d(dst, map, bar_full(stage), 0, kb * kBlock, bh);
-                tma_load_3d(dst + kPanelBytes, map, bar_full(stage), 64, kb * kBlock, bh);
+                tma_load_3d(dst, map, bar_full(stage), 0, kb * kBlock, bh, pol_kv);
+                tma_load_3d(dst + kPanelBytes, map, bar_full(stage), 64, kb * kBlock, bh, pol_kv);
                 ++issued;
             }
             // Copies in flight must land before the CTA may exit: wait for
@@ -660,7 +675,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         wv.y = pack_bf16(f[2], f[3]);
                         wv.z = pack_bf16(f[4], f[5]);
                         wv.w = pack_bf16(f[6], f[7]);
-                        o4[u] = wv;
+                        __stcs(o4 + u, wv);  // O is not re-read: stream past L2
                     }
                 }
             }
