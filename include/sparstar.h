@@ -15,6 +15,19 @@
  *      described by a forward block list (per-row count + key-block index
  *      list) without any reverse index.
  *
+ * Sources cited below:
+ *   [R-carry]  pith.science review of SparSTAR (arXiv 2608.10519), section
+ *              "What carries the argument": block-averaged q and k over
+ *              contiguous 128-token blocks, the score S_ij = tau qbar_i^T
+ *              kbar_j (Eq. 2), the block-average identity, text / Clip-1
+ *              reference retained dense, joint ranking of reference and
+ *              current blocks under the density schedule, forward-only
+ *              mask fields (FastFlex).
+ *   abstract   SparSTAR abstract (mlsanity.com/paper/2608.10519): per scale
+ *              and head, contiguous key blocks are scored from the current
+ *              query and key activations and the selected blocks run through
+ *              a forward-only sparse path.
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Tensors are [B, H, L, D] row-major, D contiguous, with no padding.
@@ -66,8 +79,8 @@ enum sparstar_status {
 
 /*
  * sparstar_block_pool — step 1, block mean pooling.
- * Passage: "block-averaged query and key vectors over contiguous 128-token
- * blocks in attention-kernel order" ([R-carry] above).
+ * Source: [R-carry] — queries and keys are averaged over contiguous 128-token
+ * blocks, taken in the order the attention kernel walks them.
  *   x     [B,H,L,D] of `dtype` (device)
  *   xbar  [B,H,ceil(L/128),D] fp32 (device, written)
  * xbar[b,h,blk,d] is the mean of the block's real tokens, summed in this
@@ -82,9 +95,9 @@ int sparstar_block_pool(const void *x, int dtype, int64_t B, int64_t H, int64_t 
 
 /*
  * sparstar_block_score — step 2a, the aggregated block score (Eq. 2).
- * Passage: "S_ij = tau qbar_i^T kbar_j ... tau = D^-1/2" and "the dot
- * product of block averages equals the average pairwise pre-softmax
- * compatibility" ([R-carry]).
+ * Source: [R-carry] — S_ij = tau qbar_i^T kbar_j with tau = D^-1/2; the dot
+ * product of two block means is the mean of the pairwise query-key dot
+ * products between the two blocks.
  *   qbar [B,H,nQB,D] fp32, kbar [B,H,nKB,D] fp32 (device)
  *   tau  fp32 scale, normally (float)(1/sqrt((double)D))
  *   S    [B,H,nQB,nKB] fp32 (device, written)
@@ -100,9 +113,9 @@ int sparstar_block_score(const float *qbar, const float *kbar, int64_t B, int64_
 /*
  * sparstar_forced_blocks — host only.  Number of leading key blocks that
  * hold at least one text or Clip-1 image-reference token:
- * ceil((text_len + image_ref_len) / 128).  Passage: text (and, for Clip 1,
- * the final image-pyramid reference) "are always retained dense"
- * ([R-carry]).  Returns -1 for negative lengths.
+ * ceil((text_len + image_ref_len) / 128).  Source: [R-carry] — text, and for
+ * Clip 1 the final image-pyramid reference, are never dropped from the
+ * attention.  Returns -1 for negative lengths.
  */
 int64_t sparstar_forced_blocks(int64_t text_len, int64_t image_ref_len);
 
@@ -117,10 +130,10 @@ int64_t sparstar_select_count(int64_t nKB, int64_t n_forced_blocks, double densi
 
 /*
  * sparstar_select — step 2b, clip-aware block Top-K into a forward-only
- * block list.  Passage: text / Clip-1 reference retained; "preceding-clip
- * reference and current-scale blocks are jointly ranked under the density
- * schedule"; FastFlex "writes only the forward mask fields and skips
- * reverse-index construction" ([R-carry]).
+ * block list.  Source: [R-carry] — text and the Clip-1 reference are kept;
+ * the remaining blocks of the preceding-clip reference and of the current
+ * scale compete in one ranking under the density budget; the mask keeps
+ * only its forward fields and builds no reverse index.
  *   S       [B,H,nQB,nKB] fp32 (device); must be finite
  *   kv_idx  [B,H,nQB,max_sel] int32 (device, written): for every row,
  *           0..nF-1, then the chosen candidates in ascending order, then -1
@@ -136,9 +149,8 @@ int sparstar_select(const float *S, int64_t B, int64_t H, int64_t nQB, int64_t n
 
 /*
  * sparstar_attn_fwd — step 3, forward attention over the listed tiles.
- * Passage: SparSTAR "executes the selected blocks through a forward-only
- * sparse path" (abstract); the chosen blocks run through a forward-only
- * attention ([R-carry]).
+ * Source: abstract and [R-carry] — only the selected blocks are computed,
+ * by a forward-only sparse attention.
  *   q [B,H,Lq,D], k and v [B,H,Lk,D] of `dtype` (device)
  *   tau      softmax scale (normally D^-1/2)
  *   kv_idx   [B,H,ceil(Lq/128),max_sel] int32, kv_cnt [B,H,ceil(Lq/128)]

@@ -19,8 +19,9 @@
  *              list, no reverse index).
  *   [R-core]   same review, "Extended reading notes / Core claim":
  *              block-wise Top-K recomputed at every scale and head.
- *   [R-ref]    same review, "Referee Report", minor comment 5: "Block-wise
- *              Top-K" and "Fresh aggregated-QK" are one mechanism.
+ *   [R-ref]    same review, "Referee Report", minor comment 5: the block-wise
+ *              Top-K of one figure and the fresh aggregated-QK selection of
+ *              one table are the same mechanism.
  *   [R-abs]    SparSTAR abstract (mlsanity.com/paper/2608.10519): scores
  *              contiguous key blocks per scale and head from the current
  *              query and key activations; executes selected blocks through
@@ -94,8 +95,8 @@ static int64_t orc_nblocks(int64_t L) { return (L + ORC_BLOCK - 1) / ORC_BLOCK; 
 /* ------------------------------------------------------- block structure */
 
 /* Forced blocks: every key block that holds at least one text token or one
- * Clip-1 image-reference token ([R-carry]: these are "always retained
- * dense", so no forced token may be dropped).  Keys are ordered
+ * Clip-1 image-reference token ([R-carry]: text and the Clip-1 reference
+ * are never dropped, so no forced token may be).  Keys are ordered
  * [text | image_ref | ref | cur], so the forced tokens are the prefix
  * 0 .. text_len + image_ref_len - 1. */
 int64_t orc_forced_blocks(int64_t text_len, int64_t image_ref_len)
