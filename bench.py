@@ -331,26 +331,55 @@ def run_gpu(args, world, rank, local):
     if int(status.item()) != 0:
         raise SystemExit("attention kernel status %#x" % int(status.item()))
 
-    # end to end through the C ABI from pinned host buffers
+    # End to end through the C ABI from pinned host buffers.  Every step
+    # copies its Q, K, V host->device and its O device->host inside the
+    # timed region.  The copies run on their own streams with double-buffered
+    # device inputs and outputs, so step s+1's upload and step s-1's download
+    # overlap step s's compute (PCIe is full duplex).
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    out_h = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+    qb = [qd, qd.clone()]
+    kbuf = [kd, kd.clone()]
+    vb = [vd, vd.clone()]
+    ob = [out, torch.empty_like(out)]
+    s_up = torch.cuda.Stream(device)
+    s_down = torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    up_done, comp_done, down_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world, device)
     torch.cuda.synchronize(device)
     e0.record(stream)
-    for _ in range(args.steps):
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        sp.sparstar_forward(qd, kd, vd, w.text, w.image_ref, w.ref, w.cur, w.density,
-                            workspace=ws, out=out, lse=lse, status=status, stream=stream)
-        out_h.copy_(out, non_blocking=True)
+    s_up.wait_event(e0)
+    s_down.wait_event(e0)
+    for step_i in range(args.steps):
+        b = step_i % 2
+        if step_i >= 2:
+            s_up.wait_event(comp_done[b])      # buffer b's previous compute has read it
+        with torch.cuda.stream(s_up):
+            qb[b].copy_(qh, non_blocking=True)
+            kbuf[b].copy_(kh, non_blocking=True)
+            vb[b].copy_(vh, non_blocking=True)
+            up_done[b].record(s_up)
+        stream.wait_event(up_done[b])
+        if step_i >= 2:
+            stream.wait_event(down_done[b])    # out[b] of step-2 has been read back
+        sp.sparstar_forward(qb[b], kbuf[b], vb[b], w.text, w.image_ref, w.ref, w.cur, w.density,
+                            workspace=ws, out=ob[b], lse=lse, status=status, stream=stream)
+        comp_done[b].record(stream)
+        s_down.wait_event(comp_done[b])
+        with torch.cuda.stream(s_down):
+            out_h[b].copy_(ob[b], non_blocking=True)
+            down_done[b].record(s_down)
+    stream.wait_event(down_done[(args.steps - 1) % 2])
+    if args.steps >= 2:
+        stream.wait_event(down_done[args.steps % 2])
     e1.record(stream)
     torch.cuda.synchronize(device)
     barrier(world, device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / args.steps
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = out_h[0].numel() * out_h[0].element_size()
 
     if rank != 0:
         return
