@@ -381,6 +381,8 @@ def run_gpu(args, world, rank, local):
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = out_h[0].numel() * out_h[0].element_size()
 
+    dense = dense_comparison(sp, w, qd, kd, vd, tau, per["attn"], stream) if args.dense else None
+
     if rank != 0:
         return
     peaks, peaks_src = read_peaks()
@@ -415,10 +417,43 @@ def run_gpu(args, world, rank, local):
         "clocks": clk.summary(),
         "flops_per_step_per_gpu": flops,
     }
+    if dense is not None:
+        line["dense_comparison"] = dense
     if world == 1 and not args.no_cpu_baseline:
         qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
         line["cpu_baseline"] = cpu_baseline(w, qn, kn, vn, flops)
     print(json.dumps(line), flush=True)
+
+
+def dense_comparison(sp, w, qd, kd, vd, tau, sparse_attn_ms, stream, reps=3):
+    """Context for the sparse operator's speed: the same scale with every
+    key block listed (this library's kernel at density 1) and torch's
+    scaled_dot_product_attention on the same tensors."""
+    nKB = w.nKB
+    idx = torch.arange(nKB, device=qd.device, dtype=torch.int32).expand(w.B, w.H, w.nQB, nKB)
+    idx = idx.contiguous()
+    cnt = torch.full((w.B, w.H, w.nQB), nKB, device=qd.device, dtype=torch.int32)
+    out = torch.empty_like(qd)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ours = timed(lambda: sp.sparstar_attn_fwd(qd, kd, vd, idx, cnt, tau, out, None,
+                                              want_lse=False, stream=stream))
+    dense_flops = 4.0 * w.D * w.Lq * w.Lk * w.B * w.H
+    sdpa = timed(lambda: torch.nn.functional.scaled_dot_product_attention(qd, kd, vd))
+    return {"ours_density1_ms": ours, "ours_density1_tflops": dense_flops / (ours * 1e-3) / 1e12,
+            "sdpa_ms": sdpa, "sdpa_tflops": dense_flops / (sdpa * 1e-3) / 1e12,
+            "sparse_attn_ms": sparse_attn_ms, "speedup_vs_sdpa": sdpa / sparse_attn_ms,
+            "speedup_vs_ours_dense": ours / sparse_attn_ms}
 
 
 def main(argv=None):
@@ -431,6 +466,8 @@ def main(argv=None):
     ap.add_argument("--ref-rows", type=int, default=256,
                     help="query rows per sampled step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", dest="dense", action="store_false",
+                    help="skip the dense comparison point (density 1 and torch SDPA)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
