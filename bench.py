@@ -273,6 +273,40 @@ def workload_config(w, world):
 
 # --------------------------------------------------------------- GPU arm
 
+def front_end_summary(w, per, peaks, clocks):
+    """Rooflines of the selection kernels.  Pooling is HBM-bound: bytes = the
+    Q and K reads + the mean writes.  The score is a fixed-order fp32 FMA
+    product (2 * D flops per block pair): in the fused kernel it runs from
+    shared memory and is bound by the FP32 pipes, peak = 148 SMs x 128 lanes
+    x 2 flops x the SM clock; in the separate chain its S write and the
+    select's S read go to memory."""
+    esz = 2 if w.dtype == "bf16" else 4
+    bh = w.B * w.H
+    pool_bytes = ((w.Lq + w.Lk) * w.D * esz + (w.nQB + w.nKB) * w.D * 4) * bh
+    score_flops = 2.0 * w.D * w.nQB * w.nKB * bh
+    s_bytes = w.nQB * w.nKB * 4 * bh
+    pool_ms = per["pool_qk"] if "pool_qk" in per else per["pool_q"] + per["pool_k"]
+    pool_gbs = pool_bytes / (pool_ms * 1e-3) / 1e9
+    out = {"pool": {"ms": pool_ms, "bytes": pool_bytes, "gbs": pool_gbs,
+                    "frac_of_hbm": pool_gbs / peaks["hbm_gbs"], "bound": "hbm"}}
+    mhz = clocks.get("sm_max_mhz") or 1965.0
+    fp32_peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    if "score_select" in per:
+        ms = per["score_select"]
+        tf = score_flops / (ms * 1e-3) / 1e12
+        out["score_select"] = {"ms": ms, "fp32_tflops": tf, "bound": "alu",
+                               "peak_fp32_tflops": fp32_peak, "frac": tf / fp32_peak,
+                               "s_bytes_kept_on_chip": s_bytes}
+    else:
+        score_bytes = (w.nQB + w.nKB) * w.D * 4 * bh + s_bytes
+        out["score"] = {"ms": per["score"], "bytes": score_bytes,
+                        "gbs": score_bytes / (per["score"] * 1e-3) / 1e9,
+                        "fp32_tflops": score_flops / (per["score"] * 1e-3) / 1e12}
+        out["select"] = {"ms": per["select"], "bytes": s_bytes,
+                         "gbs": s_bytes / (per["select"] * 1e-3) / 1e9}
+    return out
+
+
 def run_gpu(args, world, rank, local):
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
@@ -289,47 +323,90 @@ def run_gpu(args, world, rank, local):
     status = torch.zeros(1, dtype=torch.int32, device=device)
     tau = sp.default_tau(w.D)
     stream = torch.cuda.current_stream(device)
-    names = ["pool_q", "pool_k", "score", "select", "attn"]
+    sep_names = ["pool_q", "pool_k", "score", "select", "attn"]
+    fused_names = ["pool_qk", "score_select", "attn"]
 
-    def step(ev=None):
-        if ev: ev[0].record(stream)
-        sp.sparstar_block_pool(qd, ws.qbar, stream=stream)
-        if ev: ev[1].record(stream)
-        sp.sparstar_block_pool(kd, ws.kbar, stream=stream)
-        if ev: ev[2].record(stream)
-        sp.sparstar_block_score(ws.qbar, ws.kbar, tau, ws.S, stream=stream)
-        if ev: ev[3].record(stream)
+    # The separate chain: five launches, S in device memory.
+    def step_separate(st, ev=None):
+        if ev: ev[0].record(st)
+        sp.sparstar_block_pool(qd, ws.qbar, stream=st)
+        if ev: ev[1].record(st)
+        sp.sparstar_block_pool(kd, ws.kbar, stream=st)
+        if ev: ev[2].record(st)
+        sp.sparstar_block_score(ws.qbar, ws.kbar, tau, ws.S, stream=st)
+        if ev: ev[3].record(st)
         sp.sparstar_select(ws.S, ws.n_forced, w.density, kv_idx=ws.kv_idx, kv_cnt=ws.kv_cnt,
-                           stream=stream)
-        if ev: ev[4].record(stream)
-        sp.sparstar_attn_fwd(qd, kd, vd, ws.kv_idx, ws.kv_cnt, tau, out, lse, status,
-                             stream=stream)
-        if ev: ev[5].record(stream)
+                           stream=st)
+        if ev: ev[4].record(st)
+        sp.sparstar_attn_fwd(qd, kd, vd, ws.kv_idx, ws.kv_cnt, tau, out, lse, status, stream=st)
+        if ev: ev[5].record(st)
 
+    # The fused chain (the timed step): three launches, S never in memory.
+    def step_fused(st, ev=None):
+        if ev: ev[0].record(st)
+        sp.sparstar_block_pool_qk(qd, kd, ws.qbar, ws.kbar, stream=st)
+        if ev: ev[1].record(st)
+        sp.sparstar_score_select(ws.qbar, ws.kbar, ws.n_forced, w.density, tau,
+                                 kv_idx=ws.kv_idx, kv_cnt=ws.kv_cnt, stream=st)
+        if ev: ev[2].record(st)
+        sp.sparstar_attn_fwd(qd, kd, vd, ws.kv_idx, ws.kv_cnt, tau, out, lse, status, stream=st)
+        if ev: ev[3].record(st)
+
+    fused = args.chain == "fused"
+    step, names = (step_fused, fused_names) if fused else (step_separate, sep_names)
     for _ in range(args.warmup):
-        step()
+        step(stream)
     torch.cuda.synchronize(device)
     if int(status.item()) != 0:
         raise SystemExit("attention kernel status %#x" % int(status.item()))
     flops = attention_flops(ws.kv_idx.cpu().numpy(), ws.kv_cnt.cpu().numpy(), w.Lq, w.Lk, w.D)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world, device)
-    torch.cuda.synchronize(device)
-    with ClockSampler(local) as clk:
-        t0.record(stream)
-        for s in range(args.steps):
-            step(evs[s])
-        t1.record(stream)
+    def timed_steps(step_fn, n_names, use_graph):
+        """K steps bracketed by events, per-kernel events inside.  With
+        use_graph the K steps are captured into one CUDA graph (per-kernel
+        events as external record nodes) and the timed region is its single
+        replay, bracketed by events on the launching stream."""
+        evs = [[torch.cuda.Event(enable_timing=True, external=use_graph)
+                for _ in range(n_names + 1)] for _ in range(args.steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        graph = None
+        if use_graph:
+            graph = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(device)
+            cap.wait_stream(stream)
+            with torch.cuda.stream(cap), torch.cuda.graph(graph, stream=cap):
+                for s_i in range(args.steps):
+                    step_fn(cap, evs[s_i])
+            stream.wait_stream(cap)
+            graph.replay()  # upload; not timed
+            torch.cuda.synchronize(device)
+        barrier(world, device)
         torch.cuda.synchronize(device)
-    barrier(world, device)
-    total_ms = max_over_ranks(t0.elapsed_time(t1), world, device)
-    ms_per_step = total_ms / args.steps
-    per = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps
-           for i, n in enumerate(names)}
+        with ClockSampler(local) as clk_:
+            t0.record(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                for s_i in range(args.steps):
+                    step_fn(stream, evs[s_i])
+            t1.record(stream)
+            torch.cuda.synchronize(device)
+        barrier(world, device)
+        total = max_over_ranks(t0.elapsed_time(t1), world, device)
+        per_ = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(n_names)]
+        del graph
+        return total / args.steps, per_, clk_
+
+    ms_per_step, per_list, clk = timed_steps(step, len(names), fused and args.graph)
+    per = dict(zip(names, per_list))
     if int(status.item()) != 0:
         raise SystemExit("attention kernel status %#x" % int(status.item()))
+    # The other chain, eager, for comparison (same buffers, same results).
+    other_step, other_names = (step_separate, sep_names) if fused else (step_fused, fused_names)
+    other_step(stream)
+    other_ms, other_list, _ = timed_steps(other_step, len(other_names), False)
+    other = {"chain": "separate" if fused else "fused", "ms_per_step": other_ms,
+             "kernel_ms": dict(zip(other_names, other_list))}
 
     # End to end through the C ABI from pinned host buffers.  Every step
     # copies its Q, K, V host->device and its O device->host inside the
@@ -364,8 +441,9 @@ def run_gpu(args, world, rank, local):
         stream.wait_event(up_done[b])
         if step_i >= 2:
             stream.wait_event(down_done[b])    # out[b] of step-2 has been read back
-        sp.sparstar_forward(qb[b], kbuf[b], vb[b], w.text, w.image_ref, w.ref, w.cur, w.density,
-                            workspace=ws, out=ob[b], lse=lse, status=status, stream=stream)
+        fwd = sp.sparstar_forward_fused if fused else sp.sparstar_forward
+        fwd(qb[b], kbuf[b], vb[b], w.text, w.image_ref, w.ref, w.cur, w.density, workspace=ws,
+            out=ob[b], lse=lse, status=status, stream=stream)
         comp_done[b].record(stream)
         s_down.wait_event(comp_done[b])
         with torch.cuda.stream(s_down):
@@ -388,15 +466,11 @@ def run_gpu(args, world, rank, local):
     peaks, peaks_src = read_peaks()
     value = job_throughput(flops, ms_per_step, world)
     attn_tflops = flops / (per["attn"] * 1e-3) / 1e12
-    esz = 2 if w.dtype == "bf16" else 4
-    pool_bytes = ((w.Lq + w.Lk) * w.D * esz + (w.nQB + w.nKB) * w.D * 4) * w.B * w.H
-    score_bytes = ((w.nQB + w.nKB) * w.D * 4 + w.nQB * w.nKB * 4) * w.B * w.H
-    ps_ms = per["pool_q"] + per["pool_k"] + per["score"]
-    ps_gbs = (pool_bytes + score_bytes) / (ps_ms * 1e-3) / 1e9
     traffic = None
     if ATTN_TRAFFIC["source_sha256"] == attn_source_sha256():
         traffic = ATTN_TRAFFIC["bytes_per_launch"]
-    sel_ms = per["pool_q"] + per["pool_k"] + per["score"] + per["select"]
+    front = front_end_summary(w, per, peaks, clk.summary())
+    sel_ms = sum(t for n, t in per.items() if n != "attn")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -405,15 +479,16 @@ def run_gpu(args, world, rank, local):
         "attn_ms": per["attn"], "attn_tflops": attn_tflops,
         "attn_pct_of_bf16_peak": {"measured_burst": 100 * attn_tflops / peaks["bf16_tflops"],
                                   "datasheet_2250": 100 * attn_tflops / DATASHEET_BF16_TFLOPS},
+        "chain": args.chain, "graph": bool(fused and args.graph),
         "kernel_ms": per, "selection_share_pct": 100 * sel_ms / sum(per.values()),
-        "pool_score": {"ms": ps_ms, "gbs": ps_gbs, "frac_of_hbm": ps_gbs / peaks["hbm_gbs"]},
+        "front_end": front, "other_chain": other,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_tflops"],
                      "traffic": traffic,
                      "peak_source": "%s bf16 burst (MEASURED_PEAKS.json)" % peaks_src},
         "e2e": {"value": job_throughput(flops, e2e_ms, world), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": len(names) * args.steps,
         "clocks": clk.summary(),
         "flops_per_step_per_gpu": flops,
     }
@@ -465,6 +540,11 @@ def main(argv=None):
     ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--ref-rows", type=int, default=256,
                     help="query rows per sampled step of the reference arm")
+    ap.add_argument("--chain", choices=["fused", "separate"], default="fused",
+                    help="timed step: pool_qk + score_select + attn (fused) or the five "
+                         "separate calls; the other chain is timed eagerly beside it")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time the fused chain eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense comparison point (density 1 and torch SDPA)")

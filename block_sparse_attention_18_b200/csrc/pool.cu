@@ -12,6 +12,8 @@
 // explicit _rn intrinsics, so no contraction or reassociation can change
 // the bits.
 //
+// pool2_kernel does the same for two tensors (Q and K) in one launch.
+//
 // Memory: a warp covers 2 stripes x 16 chunks (bf16, D = 128), i.e. two
 // full 256-byte rows per load instruction; every thread keeps its 16 loads
 // in flight before the first add.  HBM-bound: bytes = L*D*esize read +
@@ -52,16 +54,13 @@ struct Vec<__nv_bfloat16> {
     }
 };
 
+// Mean of block `blk` of head `bh` of x [.., L, D] into xbar[row].
 template <typename T, int D>
-__global__ void __launch_bounds__(kStripes * (D * sizeof(T) / 16))
-pool_kernel(const T *__restrict__ x, int64_t L, int64_t nblk, float *__restrict__ xbar) {
+__device__ __forceinline__ void pool_block(const T *__restrict__ x, int64_t L, int64_t bh,
+                                           int64_t blk, int64_t row, float *__restrict__ xbar,
+                                           float (*stripe_sum)[D]) {
     constexpr int kElems = Vec<T>::kElems;
     constexpr int kChunks = D / kElems;  // 16-byte chunks per row
-    __shared__ float stripe_sum[kStripes][D];
-
-    const int64_t row = blockIdx.x;  // (bh, blk) flattened
-    const int64_t bh = row / nblk;
-    const int64_t blk = row - bh * nblk;
     const int64_t t0 = blk * kBlock;
     const int n = (int)((L - t0) < kBlock ? (L - t0) : kBlock);
 
@@ -107,6 +106,41 @@ pool_kernel(const T *__restrict__ x, int64_t L, int64_t nblk, float *__restrict_
 }
 
 template <typename T, int D>
+__global__ void __launch_bounds__(kStripes * (D * sizeof(T) / 16))
+pool_kernel(const T *__restrict__ x, int64_t L, int64_t nblk, float *__restrict__ xbar) {
+    __shared__ float stripe_sum[kStripes][D];
+    const int64_t row = blockIdx.x;  // (bh, blk) flattened
+    const int64_t bh = row / nblk;
+    pool_block<T, D>(x, L, bh, row - bh * nblk, row, xbar, stripe_sum);
+}
+
+// Q and K in one launch: CTAs [0, rows0) pool tensor 0, the rest tensor 1.
+template <typename T, int D>
+__global__ void __launch_bounds__(kStripes * (D * sizeof(T) / 16))
+pool2_kernel(const T *__restrict__ x0, int64_t L0, int64_t nblk0, float *__restrict__ out0,
+             const T *__restrict__ x1, int64_t L1, int64_t nblk1, float *__restrict__ out1,
+             int64_t rows0) {
+    __shared__ float stripe_sum[kStripes][D];
+    const bool second = blockIdx.x >= rows0;
+    const int64_t nblk = second ? nblk1 : nblk0;
+    const int64_t row = second ? blockIdx.x - rows0 : blockIdx.x;
+    const int64_t bh = row / nblk;
+    pool_block<T, D>(second ? x1 : x0, second ? L1 : L0, bh, row - bh * nblk, row,
+                     second ? out1 : out0, stripe_sum);
+}
+
+template <typename T, int D>
+cudaError_t launch2(const void *x0, int64_t L0, float *out0, const void *x1, int64_t L1,
+                    float *out1, int64_t BH, cudaStream_t s) {
+    const int64_t n0 = ceil_div(L0, kBlock), n1 = ceil_div(L1, kBlock);
+    const int threads = kStripes * (D * (int)sizeof(T) / 16);
+    pool2_kernel<T, D><<<(unsigned)(BH * (n0 + n1)), threads, 0, s>>>(
+        static_cast<const T *>(x0), L0, n0, out0, static_cast<const T *>(x1), L1, n1, out1,
+        BH * n0);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
 cudaError_t launch(const void *x, int64_t BH, int64_t L, float *xbar, cudaStream_t s) {
     const int64_t nblk = ceil_div(L, kBlock);
     const int threads = kStripes * (D * (int)sizeof(T) / 16);
@@ -116,6 +150,15 @@ cudaError_t launch(const void *x, int64_t BH, int64_t L, float *xbar, cudaStream
 }
 
 }  // namespace
+
+cudaError_t launch_pool2(const void *x0, int64_t L0, float *out0, const void *x1, int64_t L1,
+                         float *out1, int dtype, int64_t BH, int D, cudaStream_t stream) {
+    if (dtype == 0)
+        return D == 128 ? launch2<__nv_bfloat16, 128>(x0, L0, out0, x1, L1, out1, BH, stream)
+                        : launch2<__nv_bfloat16, 64>(x0, L0, out0, x1, L1, out1, BH, stream);
+    return D == 128 ? launch2<float, 128>(x0, L0, out0, x1, L1, out1, BH, stream)
+                    : launch2<float, 64>(x0, L0, out0, x1, L1, out1, BH, stream);
+}
 
 cudaError_t launch_pool(const void *x, int dtype, int64_t BH, int64_t L, int D, float *xbar,
                         cudaStream_t stream) {

@@ -56,8 +56,9 @@ SPARSTAR_API const char *sparstar_strerror(int code) {
     case SPARSTAR_EDTYPE: return "unsupported dtype code";
     case SPARSTAR_ECUDA: return "CUDA runtime error";
     case SPARSTAR_ESIZE:
-        return "buffer too small: max_sel below the selected count, or the intermediates "
-               "exceed the static arena (SPARSTAR_STATIC_ARENA_BYTES)";
+        return "size limit: max_sel below the selected count, the intermediates exceed the "
+               "static arena (SPARSTAR_STATIC_ARENA_BYTES), or nKB above "
+               "sparstar_score_select_max_nkb(D)";
     case SPARSTAR_ENODEV: return "no sm_100 device available for this call";
     default: return "unknown status";
     }
@@ -148,6 +149,49 @@ SPARSTAR_API int sparstar_attn_fwd(const void *q, const void *k, const void *v, 
                                                   kv_idx, kv_cnt, max_sel, out, lse, status, s));
 }
 
+SPARSTAR_API int sparstar_block_pool_qk(const void *q, const void *k, int dtype, int64_t B,
+                                        int64_t H, int64_t Lq, int64_t Lk, int64_t D,
+                                        float *qbar, float *kbar, void *stream) {
+    if (!dtype_ok(dtype)) return SPARSTAR_EDTYPE;
+    if (!q || !k || !qbar || !kbar || B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 ||
+        !head_dim_ok(D))
+        return SPARSTAR_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(qbar) || !aligned16(kbar))
+        return SPARSTAR_EINVAL;
+    if (Lq > kMaxTokens || Lk > kMaxTokens ||
+        B * H * (ceil_div(Lq, kBlock) + ceil_div(Lk, kBlock)) > kMaxGrid)
+        return SPARSTAR_EINVAL;
+    if (int rc = device_check()) return rc;
+    return cuda_status(sparstar::launch_pool2(q, Lq, qbar, k, Lk, kbar, dtype, B * H, (int)D,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+SPARSTAR_API int64_t sparstar_score_select_max_nkb(int64_t D) {
+    if (!head_dim_ok(D)) return -1;
+    return sparstar::score_select_max_nkb((int)D);
+}
+
+SPARSTAR_API int sparstar_score_select(const float *qbar, const float *kbar, int64_t B,
+                                       int64_t H, int64_t nQB, int64_t nKB, int64_t D, float tau,
+                                       int64_t n_forced_blocks, double density, int32_t *kv_idx,
+                                       int32_t *kv_cnt, int64_t max_sel, int32_t *status,
+                                       void *stream) {
+    if (!qbar || !kbar || !kv_idx || !kv_cnt || B <= 0 || H <= 0 || nQB <= 0 || nKB <= 0 ||
+        !head_dim_ok(D))
+        return SPARSTAR_EINVAL;
+    if (!std::isfinite(tau)) return SPARSTAR_EINVAL;
+    if (!aligned16(qbar) || !aligned16(kbar)) return SPARSTAR_EINVAL;
+    const int64_t sel = sparstar_select_count(nKB, n_forced_blocks, density);
+    if (sel < 0) return SPARSTAR_EINVAL;
+    if (max_sel < sel) return SPARSTAR_ESIZE;
+    if (nKB > sparstar::score_select_max_nkb((int)D)) return SPARSTAR_ESIZE;
+    if (sparstar::score_select_ctas(B * H, nQB) > kMaxGrid) return SPARSTAR_EINVAL;
+    if (int rc = device_check()) return rc;
+    return cuda_status(sparstar::launch_score_select(
+        qbar, kbar, B * H, nQB, nKB, (int)D, tau, n_forced_blocks, sel - n_forced_blocks, kv_idx,
+        kv_cnt, max_sel, status, static_cast<cudaStream_t>(stream)));
+}
+
 SPARSTAR_API int sparstar_forward(const void *q, const void *k, const void *v, int dtype,
                                   int64_t B, int64_t H, int64_t D, int64_t text_len,
                                   int64_t image_ref_len, int64_t ref_len, int64_t cur_len,
@@ -169,6 +213,31 @@ SPARSTAR_API int sparstar_forward(const void *q, const void *k, const void *v, i
     if ((rc = sparstar_block_pool(k, dtype, B, H, Lk, D, kbar, stream))) return rc;
     if ((rc = sparstar_block_score(qbar, kbar, B, H, nQB, nKB, D, tau, S, stream))) return rc;
     if ((rc = sparstar_select(S, B, H, nQB, nKB, nF, density, kv_idx, kv_cnt, max_sel, stream)))
+        return rc;
+    return sparstar_attn_fwd(q, k, v, dtype, B, H, Lq, Lk, D, tau, kv_idx, kv_cnt, max_sel, out,
+                             lse, status, stream);
+}
+
+SPARSTAR_API int sparstar_forward_fused(const void *q, const void *k, const void *v, int dtype,
+                                        int64_t B, int64_t H, int64_t D, int64_t text_len,
+                                        int64_t image_ref_len, int64_t ref_len, int64_t cur_len,
+                                        double density, float *qbar, float *kbar,
+                                        int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel,
+                                        void *out, float *lse, int32_t *status, void *stream) {
+    if (text_len < 0 || image_ref_len < 0 || ref_len < 0 || cur_len <= 0 || !head_dim_ok(D))
+        return SPARSTAR_EINVAL;
+    const int64_t Lq = cur_len, Lk = text_len + image_ref_len + ref_len + cur_len;
+    const int64_t nQB = ceil_div(Lq, kBlock), nKB = ceil_div(Lk, kBlock);
+    const int64_t nF = sparstar_forced_blocks(text_len, image_ref_len);
+    const float tau = (float)(1.0 / std::sqrt((double)D));
+    const int64_t sel = sparstar_select_count(nKB, nF, density);
+    if (sel < 0) return SPARSTAR_EINVAL;
+    if (max_sel < sel) return SPARSTAR_ESIZE;
+    if (nKB > sparstar::score_select_max_nkb((int)D)) return SPARSTAR_ESIZE;
+    int rc = sparstar_block_pool_qk(q, k, dtype, B, H, Lq, Lk, D, qbar, kbar, stream);
+    if (rc) return rc;
+    if ((rc = sparstar_score_select(qbar, kbar, B, H, nQB, nKB, D, tau, nF, density, kv_idx,
+                                    kv_cnt, max_sel, status, stream)))
         return rc;
     return sparstar_attn_fwd(q, k, v, dtype, B, H, Lq, Lk, D, tau, kv_idx, kv_cnt, max_sel, out,
                              lse, status, stream);

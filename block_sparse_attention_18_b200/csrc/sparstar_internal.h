@@ -15,6 +15,10 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 cudaError_t launch_pool(const void *x, int dtype, int64_t BH, int64_t L, int D, float *xbar,
                         cudaStream_t stream);
 
+// Step 1 for Q and K in one launch (same order, same results).
+cudaError_t launch_pool2(const void *x0, int64_t L0, float *out0, const void *x1, int64_t L1,
+                         float *out1, int dtype, int64_t BH, int D, cudaStream_t stream);
+
 // Step 2a: S = fl(tau * sequential-fma dot) for every block pair.
 cudaError_t launch_score(const float *qbar, const float *kbar, int64_t BH, int64_t nQB,
                          int64_t nKB, int D, float tau, float *S, cudaStream_t stream);
@@ -23,6 +27,20 @@ cudaError_t launch_score(const float *qbar, const float *kbar, int64_t BH, int64
 cudaError_t launch_select(const float *S, int64_t rows, int64_t nKB, int64_t nF, int64_t k,
                           int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel,
                           cudaStream_t stream);
+
+// Steps 2a + 2b fused: the scores of 16 query blocks kept in shared memory
+// and selected from there (S never written to global memory); same bits as
+// launch_score followed by launch_select.  nKB <= score_select_tiled_max_nkb()
+// runs the TMA-tiled kernel, larger nKB up to score_select_max_nkb(D) the
+// wide kernel; beyond that cudaErrorInvalidValue.  A timed-out TMA wait sets
+// SPARSTAR_STATUS_TIMEOUT in *status (if given) and empties the CTA's lists.
+cudaError_t launch_score_select(const float *qbar, const float *kbar, int64_t BH, int64_t nQB,
+                                int64_t nKB, int D, float tau, int64_t nF, int64_t k,
+                                int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel,
+                                int32_t *status, cudaStream_t stream);
+int64_t score_select_max_nkb(int D);
+int64_t score_select_tiled_max_nkb();
+int64_t score_select_ctas(int64_t BH, int64_t nQB);
 
 // Step 3, bf16 D=128: TMA + tcgen05 + TMEM kernel (sm_100a).
 int launch_attn_sm100(const void *q, const void *k, const void *v, int64_t BH, int64_t Lq,

@@ -44,11 +44,19 @@ def _load():
     L.sparstar_forward_static.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, f64,
                                           vp, vp, vp, vp]
     L.sparstar_forward_static.restype = i32
+    L.sparstar_block_pool_qk.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, vp, vp, vp]
+    L.sparstar_score_select.argtypes = [vp, vp, i64, i64, i64, i64, i64, f32, i64, f64, vp, vp,
+                                        i64, vp, vp]
+    L.sparstar_score_select_max_nkb.argtypes = [i64]
+    L.sparstar_score_select_max_nkb.restype = i64
+    L.sparstar_forward_fused.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, f64,
+                                         vp, vp, vp, vp, i64, vp, vp, vp, vp]
     L.sparstar_strerror.argtypes = [i32]
     L.sparstar_strerror.restype = ctypes.c_char_p
     L.sparstar_version.restype = i32
     for name in ("sparstar_block_pool", "sparstar_block_score", "sparstar_select",
-                 "sparstar_attn_fwd", "sparstar_forward"):
+                 "sparstar_attn_fwd", "sparstar_forward", "sparstar_block_pool_qk",
+                 "sparstar_score_select", "sparstar_forward_fused"):
         getattr(L, name).restype = i32
     return L
 
@@ -174,7 +182,8 @@ def sparstar_attn_fwd(q, k, v, kv_idx, kv_cnt, tau: float = None, out=None, lse=
 class Workspace:
     """Caller-owned device buffers for one scale of ``sparstar_forward``."""
 
-    def __init__(self, B, H, D, text_len, image_ref_len, ref_len, cur_len, density, device):
+    def __init__(self, B, H, D, text_len, image_ref_len, ref_len, cur_len, density, device,
+                 scores: bool = True):
         Lk = text_len + image_ref_len + ref_len + cur_len
         self.nQB, self.nKB = nblocks(cur_len), nblocks(Lk)
         self.n_forced = sparstar_forced_blocks(text_len, image_ref_len)
@@ -184,7 +193,9 @@ class Workspace:
         f32, i32 = torch.float32, torch.int32
         self.qbar = torch.empty(B, H, self.nQB, D, device=device, dtype=f32)
         self.kbar = torch.empty(B, H, self.nKB, D, device=device, dtype=f32)
-        self.S = torch.empty(B, H, self.nQB, self.nKB, device=device, dtype=f32)
+        # The fused front-end keeps the scores on chip and needs no S.
+        self.S = torch.empty(B, H, self.nQB, self.nKB, device=device, dtype=f32) \
+            if scores else None
         self.kv_idx = torch.empty(B, H, self.nQB, self.max_sel, device=device, dtype=i32)
         self.kv_cnt = torch.empty(B, H, self.nQB, device=device, dtype=i32)
 
@@ -207,6 +218,82 @@ def sparstar_forward(q, k, v, text_len, image_ref_len, ref_len, cur_len, density
                                 _ptr(ws.kbar), _ptr(ws.S), _ptr(ws.kv_idx), _ptr(ws.kv_cnt),
                                 ws.max_sel, _ptr(out), _ptr(lse), _ptr(status), _stream(stream)),
            "sparstar_forward")
+    return out, lse, ws
+
+
+def sparstar_block_pool_qk(q: torch.Tensor, k: torch.Tensor, qbar: torch.Tensor = None,
+                           kbar: torch.Tensor = None, stream=None):
+    """Block means of q and k in one launch; returns (qbar, kbar)."""
+    _dev(q, "q")
+    _dev(k, "k")
+    B, H, Lq, D = q.shape
+    Lk = k.shape[2]
+    if qbar is None:
+        qbar = torch.empty(B, H, nblocks(Lq), D, device=q.device, dtype=torch.float32)
+    if kbar is None:
+        kbar = torch.empty(B, H, nblocks(Lk), D, device=q.device, dtype=torch.float32)
+    _dev(qbar, "qbar", torch.float32)
+    _dev(kbar, "kbar", torch.float32)
+    dt = _DTYPE.get(q.dtype, -1) if k.dtype == q.dtype else -1
+    _check(lib.sparstar_block_pool_qk(_ptr(q), _ptr(k), dt, B, H, Lq, Lk, D, _ptr(qbar),
+                                      _ptr(kbar), _stream(stream)), "sparstar_block_pool_qk")
+    return qbar, kbar
+
+
+def sparstar_score_select_max_nkb(D: int) -> int:
+    return lib.sparstar_score_select_max_nkb(D)
+
+
+def sparstar_score_select(qbar: torch.Tensor, kbar: torch.Tensor, n_forced_blocks: int,
+                          density: float, tau: float = None, max_sel: int = None,
+                          kv_idx: torch.Tensor = None, kv_cnt: torch.Tensor = None, status=None,
+                          stream=None):
+    """Block scores and block Top-K in one launch (no S buffer); returns
+    (kv_idx, kv_cnt)."""
+    _dev(qbar, "qbar", torch.float32)
+    _dev(kbar, "kbar", torch.float32)
+    B, H, nQB, D = qbar.shape
+    nKB = kbar.shape[2]
+    if tau is None:
+        tau = default_tau(D)
+    if max_sel is None:
+        max_sel = kv_idx.shape[-1] if kv_idx is not None else \
+            sparstar_select_count(nKB, n_forced_blocks, density)
+        if max_sel < 0:
+            raise SparstarError(EINVAL, "sparstar_score_select")
+    if kv_idx is None:
+        kv_idx = torch.empty(B, H, nQB, max_sel, device=qbar.device, dtype=torch.int32)
+    if kv_cnt is None:
+        kv_cnt = torch.empty(B, H, nQB, device=qbar.device, dtype=torch.int32)
+    _dev(kv_idx, "kv_idx", torch.int32)
+    _dev(kv_cnt, "kv_cnt", torch.int32)
+    _check(lib.sparstar_score_select(_ptr(qbar), _ptr(kbar), B, H, nQB, nKB, D, tau,
+                                     n_forced_blocks, density, _ptr(kv_idx), _ptr(kv_cnt),
+                                     max_sel, _ptr(status), _stream(stream)),
+           "sparstar_score_select")
+    return kv_idx, kv_cnt
+
+
+def sparstar_forward_fused(q, k, v, text_len, image_ref_len, ref_len, cur_len, density,
+                           workspace: Workspace = None, out=None, lse=None, status=None,
+                           want_lse: bool = True, stream=None):
+    """The three-launch chain (pool q and k, score + select, attention) for one
+    scale on one stream; returns (out, lse, workspace).  The workspace needs
+    no S buffer."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, H, Lq, D = q.shape
+    ws = workspace or Workspace(B, H, D, text_len, image_ref_len, ref_len, cur_len, density,
+                                q.device, scores=False)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, Lq, device=q.device, dtype=torch.float32)
+    _check(lib.sparstar_forward_fused(_ptr(q), _ptr(k), _ptr(v), _DTYPE.get(q.dtype, -1), B, H,
+                                      D, text_len, image_ref_len, ref_len, cur_len, density,
+                                      _ptr(ws.qbar), _ptr(ws.kbar), _ptr(ws.kv_idx),
+                                      _ptr(ws.kv_cnt), ws.max_sel, _ptr(out), _ptr(lse),
+                                      _ptr(status), _stream(stream)), "sparstar_forward_fused")
     return out, lse, ws
 
 

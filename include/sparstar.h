@@ -220,6 +220,62 @@ int sparstar_forward_static(const void *q, const void *k, const void *v, int dty
                             int64_t ref_len, int64_t cur_len, double density, void *out,
                             float *lse, int32_t *status, void *stream);
 
+/*
+ * Fused selection front-end.  Source: [R-carry] — the block selection
+ * (pooling, scoring, Top-K) is a small cost beside the sparse attention it
+ * prepares; these calls make it three launches instead of five and keep S
+ * out of device memory.  Results are bit-identical to the separate calls:
+ * the same fixed fp32 orders, the same ranking and tie rule.
+ *
+ * sparstar_block_pool_qk — sparstar_block_pool of q (length Lq) into qbar
+ * and of k (length Lk) into kbar, in one launch.  Same arguments, layouts
+ * and errors as two sparstar_block_pool calls.
+ */
+int sparstar_block_pool_qk(const void *q, const void *k, int dtype, int64_t B, int64_t H,
+                           int64_t Lq, int64_t Lk, int64_t D, float *qbar, float *kbar,
+                           void *stream);
+
+/*
+ * sparstar_score_select — sparstar_block_score followed by sparstar_select
+ * in one launch, without the S buffer: each CTA scores 16 query blocks
+ * against every key block into shared memory and selects from there.
+ *   qbar, kbar, tau as for sparstar_block_score;
+ *   n_forced_blocks, density, kv_idx, kv_cnt, max_sel as for sparstar_select;
+ *   status   one int32 (device) that the kernel ORs SPARSTAR_STATUS_TIMEOUT
+ *            into if a copy wait gives up (the lists of that CTA's rows are
+ *            then empty: kv_cnt = 0), or NULL; the caller zeroes it.
+ * The score rows of 16 query blocks must fit in one CTA's shared memory:
+ * nKB <= sparstar_score_select_max_nkb(D) (2432 for D = 128, 2944 for
+ * D = 64, i.e. about 311k / 377k keys), else SPARSTAR_ESIZE and nothing is
+ * launched; the separate calls have no such limit.  Up to nKB = 1664 the
+ * key tiles arrive by TMA into a 4 x 4-per-thread product; larger nKB use a
+ * register-staged tiling that needs less shared memory per key block.
+ * Other errors as for the separate calls.
+ */
+int sparstar_score_select(const float *qbar, const float *kbar, int64_t B, int64_t H,
+                          int64_t nQB, int64_t nKB, int64_t D, float tau,
+                          int64_t n_forced_blocks, double density, int32_t *kv_idx,
+                          int32_t *kv_cnt, int64_t max_sel, int32_t *status, void *stream);
+
+/* Largest nKB sparstar_score_select accepts for head dim D; -1 for a bad D. */
+int64_t sparstar_score_select_max_nkb(int64_t D);
+
+/*
+ * sparstar_forward_fused — sparstar_forward over the fused front-end:
+ * sparstar_block_pool_qk, sparstar_score_select, sparstar_attn_fwd, three
+ * launches on one stream.  Same arguments as sparstar_forward without S;
+ * same results.  The whole chain is checked before anything is launched
+ * (SPARSTAR_ESIZE for max_sel < sel or nKB above the fused limit).  It
+ * calls no synchronising CUDA routine, so it can be recorded into a CUDA
+ * graph by stream capture once a first call on that device has run outside
+ * the capture.
+ */
+int sparstar_forward_fused(const void *q, const void *k, const void *v, int dtype, int64_t B,
+                           int64_t H, int64_t D, int64_t text_len, int64_t image_ref_len,
+                           int64_t ref_len, int64_t cur_len, double density, float *qbar,
+                           float *kbar, int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel,
+                           void *out, float *lse, int32_t *status, void *stream);
+
 /* Message for a status code (static storage). */
 const char *sparstar_strerror(int code);
 

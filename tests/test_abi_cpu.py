@@ -131,3 +131,33 @@ def test_no_device_is_reported_not_crashed(sp):
     assert L.sparstar_block_pool(A, 0, 1, 1, 128, 128, A, NUL) == sp.ENODEV
     assert L.sparstar_attn_fwd(A, A, A, 0, 1, 1, 128, 256, 128, 0.088, A, A, 2, A, NUL, NUL,
                                NUL) == sp.ENODEV
+
+
+def test_fused_front_end_limits_and_argument_errors(sp):
+    L = sp.lib
+    # 16 score rows of stride ceil(nKB/128)*128 floats plus the staged tiles
+    # must fit 227 KB of shared memory.
+    assert sp.sparstar_score_select_max_nkb(128) == 2432
+    assert sp.sparstar_score_select_max_nkb(64) == 2944
+    assert sp.sparstar_score_select_max_nkb(96) == -1
+    # every config of the scope table fits (largest: nKB 1158)
+    for w in synth.WORKLOADS.values():
+        assert w.nKB <= sp.sparstar_score_select_max_nkb(w.D)
+    ss = lambda nKB, max_sel=4000, D=128, dens=0.5, q=A: L.sparstar_score_select(
+        q, A, 1, 1, 4, nKB, D, 0.088, 2, dens, A, A, max_sel, NUL, NUL)
+    assert ss(2433) == sp.ESIZE
+    assert ss(10, max_sel=5) == sp.ESIZE
+    assert ss(10, dens=0.0) == sp.EINVAL
+    assert ss(10, D=32) == sp.EINVAL
+    assert ss(10, q=MIS) == sp.EINVAL
+    assert ss(10, q=NUL) == sp.EINVAL
+    assert L.sparstar_block_pool_qk(A, A, 5, 1, 1, 128, 256, 128, A, A, NUL) == sp.EDTYPE
+    assert L.sparstar_block_pool_qk(A, MIS, 0, 1, 1, 128, 256, 128, A, A, NUL) == sp.EINVAL
+    assert L.sparstar_block_pool_qk(A, A, 0, 1, 1, 0, 256, 128, A, A, NUL) == sp.EINVAL
+    assert L.sparstar_block_pool_qk(A, A, 0, 1, 1, 128, 256, 128, A, NUL, NUL) == sp.EINVAL
+    # the fused chain is checked before anything launches
+    fwd = lambda ref, max_sel, dens=0.5: L.sparstar_forward_fused(
+        A, A, A, 0, 1, 1, 128, 128, 0, ref, 256, dens, A, A, A, A, max_sel, A, NUL, NUL, NUL)
+    assert fwd(256, 2) == sp.ESIZE
+    assert fwd(256, 8, dens=2.0) == sp.EINVAL
+    assert fwd(2432 * 128, 4000) == sp.ESIZE  # nKB above the fused limit
