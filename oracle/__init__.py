@@ -54,6 +54,8 @@ def lib():
         L.orc_near_tie_gaps.argtypes = [vp, i64, i64, i64, i64, vp, vp]
         L.orc_attn_rows_f64.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64,
                                         vp, vp, i64, i64, vp, vp, vp]
+        L.orc_retained_mass_f64.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i64,
+                                            vp, vp, i64, i64, vp, vp, vp, vp, vp]
         _LIB = L
     return _LIB
 
@@ -180,6 +182,28 @@ def attn_rows_f64(q, k, v, kv_idx, kv_cnt, rows=None):
                             _ptr(kv_idx), _ptr(kv_cnt), max_sel, rows.size, _ptr(rows),
                             _ptr(out), _ptr(lse))
     return out, lse
+
+
+def retained_mass_f64(q, k, kv_idx, kv_cnt, nF, rows):
+    """Retained attention mass of the block lists and the token-wise bound at
+    the same candidate-token budget, in fp64, for the flat rows given.
+    Returns a dict of arrays: lse_dense, mass_block, mass_tok, mass_forced."""
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    code = _dtype_code(q)
+    assert _dtype_code(k) == code
+    B, H, Lq, D = q.shape
+    Lk = k.shape[2]
+    kv_idx = np.ascontiguousarray(kv_idx, np.int32)
+    kv_cnt = np.ascontiguousarray(kv_cnt, np.int32)
+    rows = np.ascontiguousarray(rows, np.int64)
+    out = {n: np.empty(rows.size, np.float64)
+           for n in ("lse_dense", "mass_block", "mass_tok", "mass_forced")}
+    lib().orc_retained_mass_f64(_ptr(q), _ptr(k), code, B, H, Lq, Lk, D, nF, _ptr(kv_idx),
+                                _ptr(kv_cnt), kv_idx.shape[-1], rows.size, _ptr(rows),
+                                _ptr(out["lse_dense"]), _ptr(out["mass_block"]),
+                                _ptr(out["mass_tok"]), _ptr(out["mass_forced"]))
+    return out
 
 
 def run_selection(q, k, text_len, image_ref_len, density):

@@ -22,6 +22,9 @@
  *   [R-ref]    same review, "Referee Report", minor comment 5: the block-wise
  *              Top-K of one figure and the fresh aggregated-QK selection of
  *              one table are the same mechanism.
+ *   [R-settle] same review, "What would settle it": replacing the block
+ *              score by the exact token-wise Top-K at the same densities is
+ *              the test of whether block aggregation costs fidelity.
  *   [R-abs]    SparSTAR abstract (mlsanity.com/paper/2608.10519): scores
  *              contiguous key blocks per scale and head from the current
  *              query and key activations; executes selected blocks through
@@ -430,5 +433,109 @@ void orc_attn_rows_f64(const void *q, const void *k, const void *v, int dtype,
         }
         free(qv);
         free(s);
+    }
+}
+
+/* ------------------------------------------- diagnostic: retained mass */
+
+static int orc_desc_double(const void *a, const void *b)
+{
+    const double x = *(const double *)a, y = *(const double *)b;
+    return (x < y) - (x > y);
+}
+
+/* Retained attention mass of a block list and the token-wise bound at the
+ * same budget, for the given flat query rows (bh * Lq + r), in fp64.
+ * [R-core]: block-wise Top-K recomputed at every scale stays close to the
+ * token-wise upper bound in retained attention mass; [R-settle]: the exact
+ * token-wise Top-K at the same densities is the comparison.  With the dense
+ * weights p_t = exp(tau q.k_t) / sum_u exp(tau q.k_u) over every key t < Lk:
+ *   lse_dense   = log sum_t exp(tau q.k_t)             (natural log);
+ *   mass_block  = sum of p_t over the tokens of the row's listed blocks;
+ *   mass_forced = sum of p_t over the tokens of blocks 0 .. nF-1;
+ *   M           = real tokens in the listed blocks j >= nF (the candidate
+ *                 budget the block list spends);
+ *   mass_tok    = mass_forced + the sum of the M largest p_t over the
+ *                 candidate tokens t >= 128 nF.
+ * Reading: the bound keeps the policy's forced blocks and spends the same
+ * number of candidate tokens freely, so mass_forced <= mass_block <=
+ * mass_tok <= 1.  List entries outside [0, nKB) are ignored, as in the
+ * attention. */
+void orc_retained_mass_f64(const void *q, const void *k, int dtype, int64_t B, int64_t H,
+                           int64_t Lq, int64_t Lk, int64_t D, int64_t nF,
+                           const int32_t *kv_idx, const int32_t *kv_cnt, int64_t max_sel,
+                           int64_t n_rows, const int64_t *rows, double *lse_dense,
+                           double *mass_block, double *mass_tok, double *mass_forced)
+{
+    (void)B;
+    (void)H;
+    const int64_t nQB = orc_nblocks(Lq);
+    const int64_t nKB = orc_nblocks(Lk);
+    const double tau = 1.0 / sqrt((double)D);
+    int64_t f_end = nF * ORC_BLOCK; /* first candidate token */
+    if (f_end > Lk) f_end = Lk;
+#pragma omp parallel
+    {
+        double *qv = (double *)malloc(sizeof(double) * (size_t)D);
+        double *s = (double *)malloc(sizeof(double) * (size_t)Lk);
+        double *cand = (double *)malloc(sizeof(double) * (size_t)(Lk - f_end + 1));
+        char *listed = (char *)malloc((size_t)nKB);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t n = 0; n < n_rows; ++n) {
+            const int64_t flat = rows[n];
+            const int64_t bh = flat / Lq;
+            const int64_t r = flat % Lq;
+            const int64_t list = bh * nQB + r / ORC_BLOCK;
+            for (int64_t d = 0; d < D; ++d)
+                qv[d] = (double)orc_load(q, dtype, (bh * Lq + r) * D + d);
+            /* every key's score, and the softmax normaliser */
+            double m = -INFINITY;
+            for (int64_t t = 0; t < Lk; ++t) {
+                double dot = 0.0;
+                for (int64_t d = 0; d < D; ++d)
+                    dot += qv[d] * (double)orc_load(k, dtype, (bh * Lk + t) * D + d);
+                s[t] = tau * dot;
+                if (s[t] > m) m = s[t];
+            }
+            double z = 0.0;
+            for (int64_t t = 0; t < Lk; ++t)
+                z += exp(s[t] - m);
+            const double lse = m + log(z);
+            /* the row's listed blocks */
+            for (int64_t j = 0; j < nKB; ++j)
+                listed[j] = 0;
+            int64_t cnt = kv_cnt[list];
+            if (cnt > max_sel) cnt = max_sel;
+            for (int64_t c = 0; c < cnt; ++c) {
+                const int64_t j = kv_idx[list * max_sel + c];
+                if (j >= 0 && j < nKB) listed[j] = 1;
+            }
+            double mb = 0.0, mf = 0.0;
+            int64_t budget = 0;
+            for (int64_t t = 0; t < Lk; ++t) {
+                const double p = exp(s[t] - lse);
+                if (listed[t / ORC_BLOCK]) {
+                    mb += p;
+                    if (t >= f_end) ++budget;
+                }
+                if (t < f_end) mf += p;
+            }
+            /* the M largest candidate weights */
+            const int64_t nc = Lk - f_end;
+            for (int64_t t = 0; t < nc; ++t)
+                cand[t] = exp(s[f_end + t] - lse);
+            qsort(cand, (size_t)nc, sizeof(double), orc_desc_double);
+            double top = 0.0;
+            for (int64_t t = 0; t < budget && t < nc; ++t)
+                top += cand[t];
+            lse_dense[n] = lse;
+            mass_block[n] = mb;
+            mass_forced[n] = mf;
+            mass_tok[n] = mf + top;
+        }
+        free(qv);
+        free(s);
+        free(cand);
+        free(listed);
     }
 }
