@@ -460,6 +460,7 @@ def run_gpu(args, world, rank, local):
     d2h = out_h[0].numel() * out_h[0].element_size()
 
     dense = dense_comparison(sp, w, qd, kd, vd, tau, per["attn"], stream) if args.dense else None
+    mass = retained_mass(sp, w, qd, kd, ws, lse, args.mass_rows) if args.mass_rows > 0 else None
 
     if rank != 0:
         return
@@ -494,10 +495,45 @@ def run_gpu(args, world, rank, local):
     }
     if dense is not None:
         line["dense_comparison"] = dense
+    if mass is not None:
+        line["retained_mass"] = mass
     if world == 1 and not args.no_cpu_baseline:
         qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
         line["cpu_baseline"] = cpu_baseline(w, qn, kn, vn, flops)
     print(json.dumps(line), flush=True)
+
+
+def retained_mass(sp, w, qd, kd, ws, lse, per_head, seed=0):
+    """Diagnostic, outside the timed region: on a seeded sample of query rows
+    (per head: the first row, the last row, and `per_head` random rows), the
+    dense attention mass the block lists keep, the forced blocks' share, and
+    the token-wise bound (the same forced blocks plus the M largest candidate
+    weights, M = the lists' candidate tokens).  Also checks that the block
+    mass equals exp(lse_sparse - lse_dense) with the attention kernel's LSE."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for bh in range(w.B * w.H):
+        r = {0, w.Lq - 1, *rng.choice(w.Lq, per_head, replace=False).tolist()}
+        rows.extend(bh * w.Lq + x for x in sorted(r))
+    rows_t = torch.tensor(rows, dtype=torch.int64, device=qd.device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    got = sp.sparstar_retained_mass(qd, kd, ws.kv_idx, ws.kv_cnt, ws.n_forced, rows_t)
+    b.record()
+    torch.cuda.synchronize()
+    mb = got["mass_block"].cpu().numpy()
+    mt = got["mass_tok"].cpu().numpy()
+    mf = got["mass_forced"].cpu().numpy()
+    from_lse = np.exp(lse.reshape(-1)[rows_t].double().cpu().numpy()
+                      - got["lse_dense"].cpu().numpy())
+    return {"rows": len(rows),
+            "sample": "per head: first row, last row and %d seeded random query rows" % per_head,
+            "mass_block_mean": float(mb.mean()), "mass_tok_mean": float(mt.mean()),
+            "mass_forced_mean": float(mf.mean()),
+            "gap_pct_mean": float(np.mean(100.0 * (mt - mb) / mt)),
+            "gap_pct_of_means": float(100.0 * (1.0 - mb.mean() / mt.mean())),
+            "lse_identity_max_rel": float(np.max(np.abs(from_lse / mb - 1.0))),
+            "ms": a.elapsed_time(b)}
 
 
 def dense_comparison(sp, w, qd, kd, vd, tau, sparse_attn_ms, stream, reps=3):
@@ -545,6 +581,9 @@ def main(argv=None):
                          "separate calls; the other chain is timed eagerly beside it")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time the fused chain eagerly instead of replaying a CUDA graph")
+    ap.add_argument("--mass-rows", type=int, default=64,
+                    help="random query rows per head for the retained-mass diagnostic "
+                         "(0 skips it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense comparison point (density 1 and torch SDPA)")

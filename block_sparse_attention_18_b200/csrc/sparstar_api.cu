@@ -242,3 +242,29 @@ SPARSTAR_API int sparstar_forward_fused(const void *q, const void *k, const void
     return sparstar_attn_fwd(q, k, v, dtype, B, H, Lq, Lk, D, tau, kv_idx, kv_cnt, max_sel, out,
                              lse, status, stream);
 }
+
+SPARSTAR_API int sparstar_retained_mass(const void *q, const void *k, int dtype, int64_t B,
+                                        int64_t H, int64_t Lq, int64_t Lk, int64_t D, float tau,
+                                        int64_t n_forced_blocks, const int32_t *kv_idx,
+                                        const int32_t *kv_cnt, int64_t max_sel,
+                                        const int64_t *rows, int64_t n_rows, float *scratch,
+                                        double *lse_dense, double *mass_block, double *mass_tok,
+                                        double *mass_forced, void *stream) {
+    if (!dtype_ok(dtype)) return SPARSTAR_EDTYPE;
+    if (!q || !k || !kv_cnt || !rows || !scratch || !lse_dense || !mass_block || !mass_tok ||
+        !mass_forced || B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 || !head_dim_ok(D) ||
+        n_rows <= 0 || max_sel < 0)
+        return SPARSTAR_EINVAL;
+    if (max_sel > 0 && !kv_idx) return SPARSTAR_EINVAL;
+    if (!std::isfinite(tau) || !aligned16(q) || !aligned16(k)) return SPARSTAR_EINVAL;
+    const int64_t nKB = ceil_div(Lk, kBlock);
+    if (n_forced_blocks < 0 || n_forced_blocks > nKB) return SPARSTAR_EINVAL;
+    if (Lq > kMaxTokens || Lk > kMaxTokens || nKB > sparstar::mass_max_nkb() ||
+        n_rows > kMaxGrid || max_sel > 0x7fffffffLL)
+        return SPARSTAR_EINVAL;
+    if (int rc = device_check()) return rc;
+    return cuda_status(sparstar::launch_retained_mass(
+        q, k, dtype, B * H, Lq, Lk, (int)D, tau, n_forced_blocks, kv_idx, kv_cnt, max_sel, rows,
+        n_rows, scratch, lse_dense, mass_block, mass_tok, mass_forced,
+        static_cast<cudaStream_t>(stream)));
+}

@@ -54,4 +54,14 @@ cudaError_t launch_attn_simt(const void *q, const void *k, const void *v, int dt
                              const int32_t *kv_idx, const int32_t *kv_cnt, int64_t max_sel,
                              void *out, float *lse, int32_t *status, cudaStream_t stream);
 
+// Diagnostic: retained attention mass of block lists and the token-wise
+// bound, one CTA per sampled row (scratch: n_rows * Lk fp32).
+cudaError_t launch_retained_mass(const void *q, const void *k, int dtype, int64_t BH, int64_t Lq,
+                                 int64_t Lk, int D, float tau, int64_t nF, const int32_t *kv_idx,
+                                 const int32_t *kv_cnt, int64_t max_sel, const int64_t *rows,
+                                 int64_t n_rows, float *scratch, double *lse_dense,
+                                 double *mass_block, double *mass_tok, double *mass_forced,
+                                 cudaStream_t stream);
+int64_t mass_max_nkb();
+
 }  // namespace sparstar

@@ -51,12 +51,14 @@ def _load():
     L.sparstar_score_select_max_nkb.restype = i64
     L.sparstar_forward_fused.argtypes = [vp, vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, f64,
                                          vp, vp, vp, vp, i64, vp, vp, vp, vp]
+    L.sparstar_retained_mass.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, f32, i64, vp, vp,
+                                         i64, vp, i64, vp, vp, vp, vp, vp, vp]
     L.sparstar_strerror.argtypes = [i32]
     L.sparstar_strerror.restype = ctypes.c_char_p
     L.sparstar_version.restype = i32
     for name in ("sparstar_block_pool", "sparstar_block_score", "sparstar_select",
                  "sparstar_attn_fwd", "sparstar_forward", "sparstar_block_pool_qk",
-                 "sparstar_score_select", "sparstar_forward_fused"):
+                 "sparstar_score_select", "sparstar_forward_fused", "sparstar_retained_mass"):
         getattr(L, name).restype = i32
     return L
 
@@ -315,3 +317,34 @@ def sparstar_forward_static(q, k, v, text_len, image_ref_len, ref_len, cur_len, 
                                        _ptr(out), _ptr(lse), _ptr(status), _stream(stream)),
            "sparstar_forward_static")
     return out, lse
+
+
+def sparstar_retained_mass(q, k, kv_idx, kv_cnt, n_forced_blocks: int, rows, tau: float = None,
+                           scratch=None, stream=None):
+    """Diagnostic: dense LSE, retained attention mass of the block lists, the
+    forced-block mass and the token-wise bound at the same candidate budget,
+    for the flat query rows given (int64 device tensor).  Returns a dict of
+    fp64 device tensors."""
+    _dev(q, "q")
+    _dev(k, "k")
+    _dev(kv_idx, "kv_idx", torch.int32)
+    _dev(kv_cnt, "kv_cnt", torch.int32)
+    _dev(rows, "rows", torch.int64)
+    B, H, Lq, D = q.shape
+    Lk = k.shape[2]
+    n = rows.numel()
+    if tau is None:
+        tau = default_tau(D)
+    if scratch is None:
+        scratch = torch.empty(n, Lk, device=q.device, dtype=torch.float32)
+    _dev(scratch, "scratch", torch.float32)
+    out = {name: torch.empty(n, device=q.device, dtype=torch.float64)
+           for name in ("lse_dense", "mass_block", "mass_tok", "mass_forced")}
+    dt = _DTYPE.get(q.dtype, -1) if k.dtype == q.dtype else -1
+    _check(lib.sparstar_retained_mass(_ptr(q), _ptr(k), dt, B, H, Lq, Lk, D, tau,
+                                      n_forced_blocks, _ptr(kv_idx), _ptr(kv_cnt),
+                                      kv_idx.shape[-1], _ptr(rows), n, _ptr(scratch),
+                                      _ptr(out["lse_dense"]), _ptr(out["mass_block"]),
+                                      _ptr(out["mass_tok"]), _ptr(out["mass_forced"]),
+                                      _stream(stream)), "sparstar_retained_mass")
+    return out

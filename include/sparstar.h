@@ -276,6 +276,43 @@ int sparstar_forward_fused(const void *q, const void *k, const void *v, int dtyp
                            float *kbar, int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel,
                            void *out, float *lse, int32_t *status, void *stream);
 
+/*
+ * sparstar_retained_mass — diagnostic: how much dense attention mass the
+ * block lists keep, and the most that any token-level choice with the same
+ * budget could keep.  Source: pith.science review of SparSTAR, "Extended
+ * reading notes / Core claim" (block-wise Top-K recomputed at every scale
+ * stays close to the token-wise upper bound in retained attention mass) and
+ * "What would settle it" (the exact token-wise Top-K at the same densities
+ * as the comparison).  Not part of the attention forward; it reads all of K
+ * for every sampled row.
+ *   q, k       [B,H,Lq,D], [B,H,Lk,D] of `dtype` (device)
+ *   tau        softmax scale (normally D^-1/2)
+ *   n_forced_blocks, kv_idx, kv_cnt, max_sel: the block lists, as written
+ *              by sparstar_select (device)
+ *   rows       [n_rows] int64 (device): flat query rows b*H*Lq + h*Lq + r;
+ *              a row outside [0, B*H*Lq) gets NaN results
+ *   scratch    [n_rows, Lk] fp32 (device, overwritten): the rows' scores
+ *   lse_dense, mass_block, mass_tok, mass_forced  [n_rows] fp64 (device,
+ *              written), for each row with dense weights
+ *              p_t = softmax_t(tau q.k_t) over every key t < Lk:
+ *                lse_dense   = log sum_t exp(tau q.k_t);
+ *                mass_block  = sum of p_t over the tokens of the listed blocks;
+ *                mass_forced = sum of p_t over the tokens of blocks 0..nF-1;
+ *                mass_tok    = mass_forced + the M largest p_t among the
+ *                              candidate tokens t >= 128 nF, where M = the
+ *                              real tokens of the listed blocks j >= nF.
+ * Scores are fp32 (q.k accumulated with fp32 FMAs), every sum fp64.
+ * mass_block also equals exp(lse_sparse - lse_dense) with the lse of
+ * sparstar_attn_fwd.  Errors: SPARSTAR_EINVAL for bad sizes or pointers,
+ * n_forced_blocks outside [0, nKB] or nKB > 2^20.
+ */
+int sparstar_retained_mass(const void *q, const void *k, int dtype, int64_t B, int64_t H,
+                           int64_t Lq, int64_t Lk, int64_t D, float tau, int64_t n_forced_blocks,
+                           const int32_t *kv_idx, const int32_t *kv_cnt, int64_t max_sel,
+                           const int64_t *rows, int64_t n_rows, float *scratch,
+                           double *lse_dense, double *mass_block, double *mass_tok,
+                           double *mass_forced, void *stream);
+
 /* Message for a status code (static storage). */
 const char *sparstar_strerror(int code);
 

@@ -161,3 +161,17 @@ def test_fused_front_end_limits_and_argument_errors(sp):
     assert fwd(256, 2) == sp.ESIZE
     assert fwd(256, 8, dens=2.0) == sp.EINVAL
     assert fwd(2432 * 128, 4000) == sp.ESIZE  # nKB above the fused limit
+
+
+def test_retained_mass_argument_errors(sp):
+    L = sp.lib
+    args = lambda **kw: [kw.get("q", A), A, kw.get("dtype", 0), 1, 1, 256, 640,  # noqa: E731
+                         kw.get("D", 128), 0.088, kw.get("nF", 1), A, A, 4, A,
+                         kw.get("n", 8), kw.get("scratch", A), A, A, A, A, NUL]
+    assert L.sparstar_retained_mass(*args(dtype=9)) == sp.EDTYPE
+    assert L.sparstar_retained_mass(*args(q=MIS)) == sp.EINVAL
+    assert L.sparstar_retained_mass(*args(D=80)) == sp.EINVAL
+    assert L.sparstar_retained_mass(*args(nF=6)) == sp.EINVAL  # nKB is 5
+    assert L.sparstar_retained_mass(*args(nF=-1)) == sp.EINVAL
+    assert L.sparstar_retained_mass(*args(n=0)) == sp.EINVAL
+    assert L.sparstar_retained_mass(*args(scratch=NUL)) == sp.EINVAL
