@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # SHA-256 of the kernel source it was taken on; reported only while the
 # source is unchanged.
 ATTN_TRAFFIC = {
-    "source_sha256": "d7aa7050d8be1c9e25e9a5c0a0ffe7526e426e75c4518817ba657c930cdeb204",
-    "bytes_per_launch": 5516284672 + 298376960,  # largest workload, one launch
+    "source_sha256": "37b6a093ac872170906ca791f118ea5a9f8d2683c93bc761b4616e26e6cc9c01",
+    "bytes_per_launch": 3547250176 + 307774464,  # largest workload, one launch
 }
 
 

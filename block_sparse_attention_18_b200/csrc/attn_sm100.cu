@@ -3,46 +3,39 @@
 // review, "What carries the argument": the selected blocks run through a
 // forward-only attention; the block list holds only forward fields).
 //
-// One CTA per (b, h, query block) in head-major order, so the CTAs that run
-// together share one head's K/V in L2.  Eleven warps, specialised:
-//   warps 0-7  softmax + epilogue.  Warp w serves TMEM lanes 32*(w%4)..+31
-//              (query rows) and half h = w/4 of each key tile (keys
-//              64h..64h+63), so every query row is owned by two threads and
-//              each SM sub-partition runs two softmax warps;
-//   warp 8     TMA producer: Q once, then K/V tiles in consumption order
-//              K0, K1, V0, K2, V1, ..., V(n-1) through a 6-stage ring;
-//   warp 9     TMEM allocation and the S = Q K^T MMAs;
-//   warp 10    the O += P V MMAs.
-// Two MMA warps, so each pays one wait/issue round per tile and the two
-// streams run side by side; the only cross-warp hazard (S_{j+2} written
-// over the buffer P_j is read from) is closed by the QK warp waiting for
-// the PV MMAs of tile j to complete.
-// TMEM (512 columns): S double buffer at columns 0 and 128 (fp32 128 x 128);
-// two O accumulators, O_0 at 256 and O_1 at 384, one per key half.  P of
-// half h (bf16, packed two per column) is written over columns 64h..64h+31
-// of the S buffer it came from (inside the columns the same thread read)
-// and feeds the second product straight from TMEM (tcgen05.mma with A in
-// tensor memory), so P never touches shared memory.
+// One CTA per (b, h, pair of query blocks 2p, 2p+1), head-major, so the CTAs
+// that run together share one head's K/V in L2.  The two query blocks, A
+// and B, have their own block lists and run as two interleaved pipelines:
+// while the softmax of one works, the tensor core multiplies for the other,
+// and the two softmax warpgroups drift half a period apart so their
+// exponentials (MUFU) and their TMEM traffic overlap.  Eleven warps:
+//   warps 0-3  softmax + epilogue of block A, warps 4-7 of block B: warp w
+//              serves TMEM lanes 32*(w%4)..+31, one query row per thread,
+//              all 128 columns of each key tile;
+//   warp 8     TMA producer: Q_A and Q_B once, then K(0), K(1), V(0),
+//              K(2), V(1), ... (each for A and B) through a 4-stage ring;
+//   warp 9     TMEM allocation and the S = Q K^T MMAs (A then B per step);
+//   warp 10    the O += P V MMAs (A then B per step).
+// TMEM (512 columns): S_A at 0, S_B at 128 (fp32 128 x 128), O_A at 256,
+// O_B at 384.  The softmax frees S_X as soon as it has read it into
+// registers, so S_X(j+1) = Q_X K(j+1)^T runs on the tensor core while the
+// softmax of tile j computes its exponentials.  P (bf16) goes to shared
+// memory as the K-major, 128-byte-swizzled A operand of O_X += P V; A and B
+// hand their P tiles over through one buffer in turn, each hand-off waiting
+// for the O += P V of the one before it (on that block's completion
+// barrier, so every parity wait targets the current or the next phase).
+// Shared memory: Q_A, Q_B, P (32 KB each) and a 4-stage K/V ring whose
+// keys run two steps ahead of its values.
 //
-// Per tile j: S_j = Q K_j^T (8 MMAs of K = 16, A = Q and B = K both
-// K-major, 128-byte swizzle), the softmax turns S_j into P_j, then
-// O_h += P_j,h V_j[64h..64h+63] for h = 0, 1 (4 MMAs each, A = P from
-// TMEM, B = V MN-major).  The MMA thread issues S_{j+1} before waiting for
-// P_j, so the tensor core computes the next scores while the softmax runs.
-//
-// Each key half runs its own online softmax (running max m_h, sum l_h,
-// accumulator O_h), so the two threads of a row never synchronise inside
-// the loop; the halves are merged once in the epilogue:
-//   M = max(m_0, m_1), O = sum_h 2^(m_h - M) O_h / sum_h 2^(m_h - M) l_h.
-// Scores are kept in log2 units (scaled by tau * log2(e)); a half only
-// rescales O_h and l_h when its tile max exceeds m_h by more than 8 (a
-// factor 256), which keeps P below 256 and makes the O rescale (a TMEM
-// round trip) rare.
+// Each row runs an online softmax in log2 units (running max m, sum l,
+// accumulator O_X in TMEM); O_X and l are rescaled only when the tile max
+// exceeds m by more than 8 (a factor 256), which keeps P below 256 and
+// makes the O rescale (a TMEM round trip) rare.
 //
 // Every wait is bounded (about two seconds of %globaltimer): on expiry the
 // CTA raises SPARSTAR_STATUS_TIMEOUT in *status, every role leaves its
 // loop, the producer waits (bounded) for its copies in flight, the MMA
-// thread drains its MMAs, and TMEM is freed before exit.
+// warps drain their MMAs, and TMEM is freed before exit.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -53,33 +46,35 @@
 namespace sparstar {
 namespace {
 
-constexpr int kHD = 128;                  // head dim
-constexpr int kStages = 6;                // K/V ring depth
+constexpr int kHD = 128;                      // head dim
+constexpr int kStages = 4;                    // K/V ring depth
 constexpr int kTileBytes = kBlock * kHD * 2;  // 32 KB: one Q, K or V tile
 constexpr int kPanelBytes = kTileBytes / 2;   // 16 KB: 128 rows x 64 columns
-constexpr int kSoftmaxThreads = 256;  // warps 0-7
+constexpr int kSoftmaxThreads = 256;          // warps 0-7 (128 per query block)
 constexpr int kThreads = kSoftmaxThreads + 96;
 constexpr int kProducerWarp = 8, kMmaWarp = 9, kPvWarp = 10;
 constexpr uint32_t kTmemCols = 512;
-__host__ __device__ constexpr uint32_t col_s(int b) { return (b & 1) ? 128u : 0u; }  // S buffers
-__host__ __device__ constexpr uint32_t col_o(int h) { return h ? 384u : 256u; }  // O_0, O_1
+__host__ __device__ constexpr uint32_t col_s(int x) { return x ? 128u : 0u; }  // S_A, S_B
+__host__ __device__ constexpr uint32_t col_o(int x) { return x ? 384u : 256u; }  // O_A, O_B
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
-constexpr int kOffQ = 0;
-constexpr int kOffStage = kTileBytes;
+constexpr int kOffQ = 0;                          // Q_A, then Q_B
+constexpr int kOffP = 2 * kTileBytes;             // P (bf16, K-major, swizzled), A and B in turn
+constexpr int kOffStage = 3 * kTileBytes;
 constexpr int kOffBar = kOffStage + kStages * kTileBytes;
 struct Bars {
     uint64_t q_full;
     uint64_t st_full[kStages];
     uint64_t st_empty[kStages];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t pv_done[2];
+    uint64_t s_full[2];   // per query block
+    uint64_t s_free[2];
+    uint64_t p_full[2][2];   // [block][half of P]: keys 64h .. 64h+63 written
+    uint64_t pv_half[2][2];  // [block][half]: O += P_half V_half complete
     uint64_t drain;
     uint32_t tmem_base;
     int32_t abort_flag;
-    int32_t n_valid;
+    int32_t n_valid[2];
 };
 constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 1024;  // + alignment slack
 
@@ -240,14 +235,6 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -267,14 +254,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "%28, %29, %30, %31}, [%32];"
         : SPX_R8(0), SPX_R8(8), SPX_R8(16), SPX_R8(24)
         : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-        "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
-        "%27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        SPX_W8(0), SPX_W8(8), SPX_W8(16), SPX_W8(24)
-        : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -330,15 +309,47 @@ __device__ __forceinline__ int next_valid(const int32_t *list, int cnt, int &cur
     return 0;  // unreachable when the caller counts valid entries first
 }
 
+// 8 consecutive fp32 columns of this thread's TMEM lane (the rare O rescale
+// uses these narrow chunks so that a full row of scores stays in registers).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+                   "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
+// Producer order: K(0), K(1), then for s = 0, 1, ...: V(s), K(s+2), where
+// K(j) stands for K_A(j), K_B(j) and V(j) for V_A(j), V_B(j), each present
+// while j is below that block's tile count.  Keys run two steps ahead of
+// values, so the next S products never wait for a value tile's slot.
+// C(m) counts the tiles of steps before m; the ring index of each tile is
+// the number of tiles the producer loads before it.
+__device__ __forceinline__ int steps_before(int m, int nA, int nB) {
+    m = m < 0 ? 0 : m;
+    return (m < nA ? m : nA) + (m < nB ? m : nB);
+}
+__device__ __forceinline__ int slot_k(int x, int j, int nA, int nB) {
+    return steps_before(j, nA, nB) + steps_before(j - 1, nA, nB) + ((x == 1 && j < nA) ? 1 : 0);
+}
+__device__ __forceinline__ int slot_v(int x, int j, int nA, int nB) {
+    return steps_before(j + 2, nA, nB) + steps_before(j, nA, nB) + ((x == 1 && j < nA) ? 1 : 0);
+}
 // ------------------------------------------------------------------ kernel
 
-__global__ void __launch_bounds__(kThreads, 1)
-attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, int Lq, int Lk, int nQB, int nKB,
-                  float tau, const int32_t *__restrict__ kv_idx,
-                  const int32_t *__restrict__ kv_cnt, int max_sel,
-                  __nv_bfloat16 *__restrict__ out, float *__restrict__ lse,
-                  int32_t *__restrict__ status) {
+__global__ void __maxnreg__(168)
+attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, int Lq, int Lk, int nQB, int nKB,
+                       int nPair, float tau, const int32_t *__restrict__ kv_idx,
+                       const int32_t *__restrict__ kv_cnt, int max_sel,
+                       __nv_bfloat16 *__restrict__ out, float *__restrict__ lse,
+                       int32_t *__restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -347,21 +358,29 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     volatile int32_t *abort_flag = &bars->abort_flag;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x / nQB;
-    const int qb = blockIdx.x % nQB;
-    const int32_t *list = kv_idx + (int64_t)blockIdx.x * max_sel;
+    const int bh = blockIdx.x / nPair;
+    const int qb0 = 2 * (blockIdx.x % nPair);  // query block A; B = qb0 + 1
+    const bool hasB = qb0 + 1 < nQB;
+    // Lists and counts of A (x = 0) and B (x = 1); an absent B has none.
+    const int64_t rowA = (int64_t)bh * nQB + qb0;
+    const int32_t *listA = kv_idx + rowA * max_sel;
+    const int32_t *listB = kv_idx + (hasB ? rowA + 1 : rowA) * max_sel;
+    int cntA = __ldg(kv_cnt + rowA), cntB = hasB ? __ldg(kv_cnt + rowA + 1) : 0;
+    cntA = cntA < 0 ? 0 : (cntA > max_sel ? max_sel : cntA);
+    cntB = cntB < 0 ? 0 : (cntB > max_sel ? max_sel : cntB);
 
     const uint32_t bar_q = smem_addr(&bars->q_full);
     auto bar_full = [&](int s) { return smem_addr(&bars->st_full[s]); };
     auto bar_empty = [&](int s) { return smem_addr(&bars->st_empty[s]); };
-    auto bar_s = [&](int b) { return smem_addr(&bars->s_full[b]); };
-    auto bar_p = [&](int b) { return smem_addr(&bars->p_full[b]); };
-    auto bar_pv = [&](int b) { return smem_addr(&bars->pv_done[b]); };
+    auto bar_s = [&](int x) { return smem_addr(&bars->s_full[x]); };
+    auto bar_sfree = [&](int x) { return smem_addr(&bars->s_free[x]); };
+    auto bar_p = [&](int x, int h) { return smem_addr(&bars->p_full[x][h]); };
+    auto bar_ph = [&](int x, int h) { return smem_addr(&bars->pv_half[x][h]); };
+    // the whole O += P V of a block (its second half completes last)
+    auto bar_pv = [&](int x) { return smem_addr(&bars->pv_half[x][1]); };
     const uint32_t bar_drain = smem_addr(&bars->drain);
 
-    // ---- set-up: barriers, valid-entry count, TMEM
-    int cnt = __ldg(kv_cnt + blockIdx.x);
-    cnt = cnt < 0 ? 0 : (cnt > max_sel ? max_sel : cnt);
+    // ---- set-up: barriers, valid-entry counts, TMEM
     if (warp == kProducerWarp) {
         if (lane == 0) {
             mbar_init(bar_q, 1);
@@ -369,10 +388,13 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 mbar_init(bar_full(s), 1);
                 mbar_init(bar_empty(s), 1);
             }
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(bar_s(b), 1);
-                mbar_init(bar_p(b), kSoftmaxThreads);
-                mbar_init(bar_pv(b), 1);
+            for (int x = 0; x < 2; ++x) {
+                mbar_init(bar_s(x), 1);
+                mbar_init(bar_sfree(x), kSoftmaxThreads / 2);
+                for (int h = 0; h < 2; ++h) {
+                    mbar_init(bar_p(x, h), kSoftmaxThreads / 2);
+                    mbar_init(bar_ph(x, h), 1);
+                }
             }
             mbar_init(bar_drain, 2);  // one commit from each MMA warp
             bars->abort_flag = 0;
@@ -381,17 +403,22 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)));
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmV)));
         }
-        int nv = 0;
-        for (int c = lane; c < cnt; c += 32) {
-            const int j = __ldg(list + c);
-            if (j >= 0 && j < nKB)
-                ++nv;
-            else if (status)
-                atomicOr(status, SPARSTAR_STATUS_BAD_INDEX);
-        }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, o);
-        if (lane == 0) bars->n_valid = nv;
+        for (int x = 0; x < 2; ++x) {
+            const int32_t *lx = x ? listB : listA;
+            const int cx = x ? cntB : cntA;
+            int nv = 0;
+            for (int c = lane; c < cx; c += 32) {
+                const int j = __ldg(lx + c);
+                if (j >= 0 && j < nKB)
+                    ++nv;
+                else if (status)
+                    atomicOr(status, SPARSTAR_STATUS_BAD_INDEX);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, o);
+            if (lane == 0) bars->n_valid[x] = nv;
+        }
     } else if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_addr(&bars->tmem_base)),
@@ -403,115 +430,150 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const int n = bars->n_valid;
+    const int nA = bars->n_valid[0], nB = bars->n_valid[1];
+    const int nmax = nA > nB ? nA : nB;
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------------ TMA producer
-        if (lane == 0 && n > 0) {
-            const uint32_t sQ = base + kOffQ;
+        if (lane == 0 && nmax > 0) {
             const uint64_t pol_q = policy_evict_first(), pol_kv = policy_evict_normal();
-            mbar_expect_tx(bar_q, kTileBytes);
-            tma_load_3d(sQ, &tmQ, bar_q, 0, qb * kBlock, bh, pol_q);
-            tma_load_3d(sQ + kPanelBytes, &tmQ, bar_q, 64, qb * kBlock, bh, pol_q);
-            int curK = 0, curV = 0;
-            int issued = 0;
+            const int nq = nB > 0 ? 2 : 1;  // Q_B only when B has work
+            mbar_expect_tx(bar_q, nq * kTileBytes);
+            for (int x = 0; x < nq; ++x) {
+                const uint32_t sQ = base + kOffQ + x * kTileBytes;
+                const int qrow = (x == 0 ? qb0 : qb0 + 1) * kBlock;
+                tma_load_3d(sQ, &tmQ, bar_q, 0, qrow, bh, pol_q);
+                tma_load_3d(sQ + kPanelBytes, &tmQ, bar_q, 64, qrow, bh, pol_q);
+            }
+            int curKA = 0, curKB = 0, curVA = 0, curVB = 0;
+            int e = 0;
             bool ok = true;
-            for (int e = 0; e < 2 * n && ok; ++e) {
-                const int stage = e % kStages;
-                const uint32_t ph = (uint32_t)(e / kStages) & 1u;
-                if (!wait1(bar_empty(stage), ph ^ 1u, abort_flag, status)) {
-                    ok = false;
-                    break;
+            // Groups K(0), K(1), V(0), K(2), V(1), K(3), ...: group g > 0
+            // is K((g+1)/2) when odd, V(g/2-1) when even.
+            for (int g = 0; g <= 2 * nmax && ok; ++g) {
+                const bool is_v = g > 0 && (g & 1) == 0;
+                const int j = g == 0 ? 0 : (is_v ? g / 2 - 1 : (g + 1) / 2);
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (j >= (x == 0 ? nA : nB)) continue;
+                    const int stage = e % kStages;
+                    if (!wait1(bar_empty(stage), ((uint32_t)(e / kStages) & 1u) ^ 1u, abort_flag,
+                               status)) {
+                        ok = false;
+                        break;
+                    }
+                    const int32_t *lx = x ? listB : listA;
+                    const int cx = x ? cntB : cntA;
+                    int &cr = is_v ? (x ? curVB : curVA) : (x ? curKB : curKA);
+                    const int kb = next_valid(lx, cx, cr, nKB);
+                    const uint32_t dst = base + kOffStage + stage * kTileBytes;
+                    const CUtensorMap *map = is_v ? &tmV : &tmK;
+                    mbar_expect_tx(bar_full(stage), kTileBytes);
+                    tma_load_3d(dst, map, bar_full(stage), 0, kb * kBlock, bh, pol_kv);
+                    tma_load_3d(dst + kPanelBytes, map, bar_full(stage), 64, kb * kBlock, bh,
+                                pol_kv);
+                    ++e;
                 }
-                const bool is_v = (e == 2 * n - 1) || (e > 0 && (e & 1) == 0);
-                const int kb = is_v ? next_valid(list, cnt, curV, nKB)
-                                    : next_valid(list, cnt, curK, nKB);
-                const uint32_t dst = base + kOffStage + stage * kTileBytes;
-                const CUtensorMap *map = is_v ? &tmV : &tmK;
-                mbar_expect_tx(bar_full(stage), kTileBytes);
-                tma_load_3d(dst, map, bar_full(stage), 0, kb * kBlock, bh, pol_kv);
-                tma_load_3d(dst + kPanelBytes, map, bar_full(stage), 64, kb * kBlock, bh, pol_kv);
-                ++issued;
             }
             // Copies in flight must land before the CTA may exit: wait for
             // Q and for the latest arming of every stage (no-ops normally).
             drain_wait(bar_q, 0);
-            const int first = issued > kStages ? issued - kStages : 0;
-            for (int e = first; e < issued; ++e)
-                drain_wait(bar_full(e % kStages), (uint32_t)(e / kStages) & 1u);
+            const int first = e > kStages ? e - kStages : 0;
+            for (int i = first; i < e; ++i)
+                drain_wait(bar_full(i % kStages), (uint32_t)(i / kStages) & 1u);
         }
     } else if (warp == kMmaWarp) {
         // -------------------------------------------- S = Q K^T MMA issuer
-        // The whole warp runs the control flow, so descriptors and TMEM
-        // addresses stay warp-uniform; one elected lane issues.  Descriptors
+        // Warp-uniform control flow; one elected lane issues.  Descriptors
         // are built once per operand and advanced by compile-time offsets.
-        const uint64_t dQ = desc_k_major(base + kOffQ);
-        bool ok = n > 0 && wait_warp(bar_q, 0, abort_flag, status);
-        for (int j = 0; j < n && ok; ++j) {
-            const int e = j == 0 ? 0 : 2 * j - 1;  // ring slot of K_j
-            const int stage = e % kStages;
-            if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
-                ok = false;
-                break;
-            }
-            if (j >= 2) {
-                // S buffer j&1 still holds P_{j-2} until its PV MMAs complete.
-                if (!wait_warp(bar_pv(j & 1), (uint32_t)((j - 2) >> 1) & 1u, abort_flag, status)) {
+        const uint64_t dQ0 = desc_k_major(base + kOffQ);
+        const uint64_t dQ1 = desc_k_major(base + kOffQ + kTileBytes);
+        bool ok = nmax > 0 && wait_warp(bar_q, 0, abort_flag, status);
+        for (int j = 0; j < nmax && ok; ++j) {
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                if (!ok || j >= (x == 0 ? nA : nB)) continue;
+                const int e = slot_k(x, j, nA, nB);
+                const int stage = e % kStages;
+                if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag,
+                               status)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-            }
-            const uint64_t dK = desc_k_major(base + kOffStage + stage * kTileBytes);
-            const uint32_t dS = tmem + col_s(j & 1);
-            if (elect_one()) {
-#pragma unroll
-                for (int kk = 0; kk < kHD / 16; ++kk) {
-                    const uint64_t off = (uint64_t)(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
-                    mma_ss(dS, dQ + off, dK + off, kIdescQK, kk > 0 ? 1u : 0u);
+                if (j >= 1) {
+                    // S_x is free once the softmax has read S_x(j-1).
+                    if (!wait_warp(bar_sfree(x), (uint32_t)(j - 1) & 1u, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
                 }
-                mma_commit(bar_empty(stage));
-                mma_commit(bar_s(j & 1));
+                const uint64_t dK = desc_k_major(base + kOffStage + stage * kTileBytes);
+                const uint64_t dQ = x == 0 ? dQ0 : dQ1;
+                const uint32_t dS = tmem + col_s(x);
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < kHD / 16; ++kk) {
+                        const uint64_t off =
+                            (uint64_t)(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
+                        mma_ss(dS, dQ + off, dK + off, kIdescQK, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar_empty(stage));
+                    mma_commit(bar_s(x));
+                }
+                __syncwarp();
             }
-            __syncwarp();
         }
         // Drain: every MMA this warp issued completes before TMEM is freed.
-        if (n > 0) {
+        if (nmax > 0) {
             if (elect_one()) mma_commit(bar_drain);
             __syncwarp();
         }
     } else if (warp == kPvWarp) {
         // ---------------------------------------------- O += P V MMA issuer
-        bool ok = n > 0;
-        for (int jj = 0; jj < n && ok; ++jj) {
-            if (!wait_warp(bar_p(jj & 1), (uint32_t)(jj >> 1) & 1u, abort_flag, status)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();  // orders the softmax's tcgen05.st of P before the MMA
-            const int e = jj == n - 1 ? 2 * n - 1 : 2 * jj + 2;  // ring slot of V_jj
-            const int stage = e % kStages;
-            if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag, status)) {
-                ok = false;
-                break;
-            }
-            const uint64_t dV = desc_mn_major(base + kOffStage + stage * kTileBytes);
-            const uint32_t aP = tmem + col_s(jj & 1);
-            const uint32_t first = jj > 0 ? 1u : 0u;
-            if (elect_one()) {
+        bool ok = nmax > 0;
+        for (int j = 0; j < nmax && ok; ++j) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
+            for (int x = 0; x < 2; ++x) {
+                if (!ok || j >= (x == 0 ? nA : nB)) continue;
+                if (!wait_warp(bar_p(x, 0), (uint32_t)j & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();  // orders an O rescale (tcgen05.st) before the MMA
+                const int e = slot_v(x, j, nA, nB);
+                const int stage = e % kStages;
+                if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag,
+                               status)) {
+                    ok = false;
+                    break;
+                }
+                const uint64_t dV = desc_mn_major(base + kOffStage + stage * kTileBytes);
+                const uint64_t dP = desc_k_major(base + kOffP);
+                const uint32_t first = j > 0 ? 1u : 0u;
+                // Each half of P (keys 64h .. 64h+63, one 16 KB panel) is
+                // multiplied as soon as it is written.
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + col_o(h), aP + 64u * h + 8u * kk,
-                               dV + (uint64_t)(((4 * h + kk) * 16 * 128) >> 4), kIdescPV,
-                               kk > 0 ? 1u : first);
-                mma_commit(bar_empty(stage));
-                mma_commit(bar_pv(jj & 1));
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 1 && !wait_warp(bar_p(x, 1), (uint32_t)j & 1u, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (elect_one()) {
+#pragma unroll
+                        for (int kq = 0; kq < 4; ++kq) {
+                            const int kk = 4 * h + kq;
+                            mma_ss(tmem + col_o(x), dP + (uint64_t)((h * kPanelBytes + kq * 32) >> 4),
+                                   dV + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV,
+                                   kk > 0 ? 1u : first);
+                        }
+                        if (h == 1) mma_commit(bar_empty(stage));
+                        mma_commit(bar_ph(x, h));
+                    }
+                    __syncwarp();
+                }
             }
-            __syncwarp();
         }
-        if (n > 0) {
+        if (nmax > 0) {
             if (elect_one()) mma_commit(bar_drain);
             __syncwarp();
             // Both MMA warps have committed to the drain barrier; its phase
@@ -520,85 +582,111 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
         __syncwarp();
     } else {
-        // ------------------------------------------ softmax + epilogue (256 thr)
+        // ------------------------------- softmax + epilogue (128 per block)
+        const int x = warp >> 2;           // query block: 0 = A, 1 = B
         const int quarter = warp & 3;      // TMEM lane quarter
-        const int half = warp >> 2;        // key half of every tile
         const int row = quarter * 32 + lane;  // TMEM lane == tile row
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t colO = col_o(half);
+        const uint32_t colS = col_s(x), colO = col_o(x);
+        const int nx = x == 0 ? nA : nB;
         const float sc = tau * 1.4426950408889634f;  // scores in log2 units
         float m_ref = -INFINITY, l = 0.0f;
         bool ok = true;
         int cur = 0;
-        for (int j = 0; j < n; ++j) {
-            const int kb = next_valid(list, cnt, cur, nKB);
-            if (!wait_warp(bar_s(j & 1), (uint32_t)(j >> 1) & 1u, abort_flag, status)) {
+        for (int j = 0; j < nx; ++j) {
+            const int kb = next_valid(x ? listB : listA, x ? cntB : cntA, cur, nKB);
+            if (!wait_warp(bar_s(x), (uint32_t)j & 1u, abort_flag, status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t colS = col_s(j & 1) + 64u * half;
-            float s[64];
+            float s[128];
             {
-                uint32_t r[2][32];
-                tmem_ld32(tmem + lane_base + colS, r[0]);
-                tmem_ld32(tmem + lane_base + colS + 32, r[1]);
-                tmem_wait_ld();
-                reg_fence(r[0]);
-                reg_fence(r[1]);
+                uint32_t r[4][32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
+                for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + colS + 32 * c, r[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) reg_fence(r[c]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
                     for (int u = 0; u < 32; ++u) s[32 * c + u] = __uint_as_float(r[c][u]);
             }
-            const int valid = Lk - kb * kBlock - 64 * half;  // keys of this half that exist
-            if (valid < 64) {
+            // S_x(j) is in registers: the next S = Q K^T may overwrite it.
+            tc_fence_before();
+            mbar_arrive(bar_sfree(x));
+            const int valid = Lk - kb * kBlock;  // keys of this tile that exist
+            if (valid < kBlock) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
+                for (int c = 0; c < kBlock; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
             float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int c = 4; c < 64; c += 8) {
+            for (int c = 4; c < kBlock; c += 8) {
 #pragma unroll
                 for (int t = 0; t < 4; ++t) mx[t] = max3f(mx[t], s[c + t], s[c + 4 + t]);
             }
             const float m_tile = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
             const float m_new = fmaxf(m_ref, m_tile);
+            bool p_free = false;  // the P buffer is free for this hand-off
             if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
                 if (j > 0) {
-                    if (!wait_warp(bar_pv((j - 1) & 1), (uint32_t)((j - 1) >> 1) & 1u, abort_flag,
-                                   status)) {
+                    if (!wait_warp(bar_pv(x), (uint32_t)(j - 1) & 1u, abort_flag, status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const float f = m_new > -INFINITY ? ex2(m_ref - m_new) : 1.0f;  // 0 if no key seen yet
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(tmem + lane_base + colO + 32 * c, r);
+                    const float f = m_new > -INFINITY ? ex2(m_ref - m_new) : 1.0f;
+#pragma unroll 1
+                    for (int c = 0; c < kHD / 8; ++c) {
+                        uint32_t r[8];
+                        tmem_ld8(tmem + lane_base + colO + 8 * c, r);
                         tmem_wait_ld();
-                        reg_fence(r);
+                        asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]),
+                                     "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
 #pragma unroll
-                        for (int u = 0; u < 32; ++u)
+                        for (int u = 0; u < 8; ++u)
                             r[u] = __float_as_uint(__uint_as_float(r[u]) * f);
-                        tmem_st32(tmem + lane_base + colO + 32 * c, r);
+                        tmem_st8(tmem + lane_base + colO + 8 * c, r);
                     }
                     tmem_wait_st();
                 }
-                if (m_new > -INFINITY) {  // a half with no key yet keeps l = 0
+                if (m_new > -INFINITY) {  // a row with no key yet keeps l = 0
                     l *= ex2(m_ref - m_new);
                     m_ref = m_new;
                 }
             }
-            // m_ref = -inf only while every key of this half so far was masked:
-            // then every p is 0 (a finite offset keeps -inf * sc + offset = -inf).
+            // m_ref = -inf only while every key so far was masked: then
+            // every p is 0 (a finite offset keeps -inf * sc + offset = -inf).
             const float neg_m = m_ref > -INFINITY ? -m_ref : 0.0f;
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[32];
+            // P (bf16) in shared memory as the K-major, 128-byte-swizzled A
+            // operand of O += P V: panel h holds keys 64h..64h+63, row r at
+            // r * 128 bytes, 16-byte chunk c (keys 8c..8c+7) at c ^ (r & 7).
+            // A and B take the one buffer in turn, in the order A(0), B(0),
+            // A(1), B(1), ... (a block past its last tile drops out): a
+            // hand-off waits for the O += P V of the hand-off before it.
+            // That one is at most one phase ahead of what this warpgroup
+            // has already seen on its barrier, so a parity wait is exact.
+            uint8_t *prow = smem + kOffP + row * 128;
+            int prev_x = -1, prev_j = -1;
+            if (x == 0) {
+                if (j >= 1) {
+                    prev_j = j - 1;
+                    prev_x = j - 1 < nB ? 1 : 0;
+                }
+            } else if (j < nA) {
+                prev_x = 0;
+                prev_j = j;
+            } else if (j >= 1) {
+                prev_x = 1;
+                prev_j = j - 1;
+            }
+            uint32_t pk[64];  // P of keys 2u, 2u+1 in pk[u]
 #pragma unroll
-            for (int u = 0; u < 32; u += 2) {
+            for (int u = 0; u < 64; u += 2) {
                 const int c = 2 * u;
                 const float p0 = ex2(fmaf(s[c], sc, neg_m));
                 const float p1 = ex2(fmaf(s[c + 1], sc, neg_m));
@@ -611,76 +699,75 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 pk[u] = pack_bf16(p0, p1);
                 pk[u + 1] = pack_bf16(p2, p3);
             }
-            tmem_st32(tmem + lane_base + colS, pk);
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar_p(j & 1));
+            // Hand P over half by half: half h waits for the previous
+            // hand-off's O += P_h V_h, is stored, and is released to the MMA
+            // warp (after the proxy fence that orders the generic-proxy
+            // stores before the tensor core's reads; the first release also
+            // orders any O rescale before the next O += P V).
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (prev_x >= 0) {
+                    p_free = wait_warp(bar_ph(prev_x, h), (uint32_t)prev_j & 1u, abort_flag, status);
+                    if (!p_free) break;
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(prow + h * kPanelBytes + ((c ^ (row & 7)) << 4)) =
+                        make_uint4(pk[32 * h + 4 * c], pk[32 * h + 4 * c + 1],
+                                   pk[32 * h + 4 * c + 2], pk[32 * h + 4 * c + 3]);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                if (h == 0) tc_fence_before();
+                mbar_arrive(bar_p(x, h));
+            }
+            if (prev_x >= 0 && !p_free) {
+                ok = false;
+                break;
+            }
         }
 
-        // ---- epilogue: merge the two halves, O / l -> bf16, LSE
-        const bool have = n > 0 && ok &&
-                          wait_warp(bar_pv((n - 1) & 1), (uint32_t)((n - 1) >> 1) & 1u, abort_flag,
-                                    status);
-        // Exchange (m, l) with the partner thread of the other half.  Every
-        // MMA has completed once the last O update has (or the CTA is
-        // aborting), so the Q tile's shared memory is free for this.
-        float *xm = reinterpret_cast<float *>(smem + kOffQ);  // [2][128]
-        float *xl = xm + 2 * kBlock;                           // [2][128]
-        xm[half * kBlock + row] = m_ref;
-        xl[half * kBlock + row] = l;
-        asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
-        const float m_o = xm[(half ^ 1) * kBlock + row];
-        const float l_o = xl[(half ^ 1) * kBlock + row];
-        const float M = fmaxf(m_ref, m_o);
-        const float a_self = m_ref > -INFINITY ? ex2(m_ref - M) : 0.0f;
-        const float a_oth = m_o > -INFINITY ? ex2(m_o - M) : 0.0f;
-        const float L = l * a_self + l_o * a_oth;
-        const float a0 = half == 0 ? a_self : a_oth;  // weight of O_0
-        const float a1 = half == 0 ? a_oth : a_self;  // weight of O_1
-
+        // ---- epilogue: O / l -> bf16, LSE
+        const bool have = nx > 0 && ok &&
+                          wait_warp(bar_pv(x), (uint32_t)(nx - 1) & 1u, abort_flag, status);
+        const int qb = qb0 + x;
         const int64_t grow = (int64_t)qb * kBlock + row;
-        const bool store = grow < Lq;
-        __nv_bfloat16 *orow = out + ((int64_t)bh * Lq + grow) * kHD + 64 * half;
-        if (n == 0) {
+        const bool store = qb < nQB && grow < Lq;
+        __nv_bfloat16 *orow = out + ((int64_t)bh * Lq + grow) * kHD;
+        if (nx == 0) {
             if (store) {
                 uint4 *o4 = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) o4[c] = make_uint4(0, 0, 0, 0);
-                if (lse && half == 0) lse[(int64_t)bh * Lq + grow] = -INFINITY;
+                for (int c = 0; c < 16; ++c) o4[c] = make_uint4(0, 0, 0, 0);
+                if (lse) lse[(int64_t)bh * Lq + grow] = -INFINITY;
             }
         } else if (have) {
             tc_fence_after();
-            const float inv = 1.0f / L;
-            const float w0 = a0 * inv, w1 = a1 * inv;
+            const float inv = 1.0f / l;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {  // output columns 64*half + 32c .. +31
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tmem + lane_base + col_o(0) + 64 * half + 32 * c, r0);
-                tmem_ld32(tmem + lane_base + col_o(1) + 64 * half + 32 * c, r1);
+            for (int c = 0; c < 4; ++c) {  // output columns 32c .. 32c+31
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + colO + 32 * c, r);
                 tmem_wait_ld();
-                reg_fence(r0);
-                reg_fence(r1);
+                reg_fence(r);
                 if (store) {
                     uint4 *o4 = reinterpret_cast<uint4 *>(orow + 32 * c);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        float f[8];
-#pragma unroll
-                        for (int t = 0; t < 8; ++t)
-                            f[t] = __uint_as_float(r0[8 * u + t]) * w0 +
-                                   __uint_as_float(r1[8 * u + t]) * w1;
                         uint4 wv;
-                        wv.x = pack_bf16(f[0], f[1]);
-                        wv.y = pack_bf16(f[2], f[3]);
-                        wv.z = pack_bf16(f[4], f[5]);
-                        wv.w = pack_bf16(f[6], f[7]);
+                        wv.x = pack_bf16(__uint_as_float(r[8 * u + 0]) * inv,
+                                         __uint_as_float(r[8 * u + 1]) * inv);
+                        wv.y = pack_bf16(__uint_as_float(r[8 * u + 2]) * inv,
+                                         __uint_as_float(r[8 * u + 3]) * inv);
+                        wv.z = pack_bf16(__uint_as_float(r[8 * u + 4]) * inv,
+                                         __uint_as_float(r[8 * u + 5]) * inv);
+                        wv.w = pack_bf16(__uint_as_float(r[8 * u + 6]) * inv,
+                                         __uint_as_float(r[8 * u + 7]) * inv);
                         __stcs(o4 + u, wv);  // O is not re-read: stream past L2
                     }
                 }
             }
-            if (store && lse && half == 0)
-                lse[(int64_t)bh * Lq + grow] = (M + log2f(L)) * 0.6931471805599453f;
+            if (store && lse)
+                lse[(int64_t)bh * Lq + grow] = (m_ref + log2f(l)) * 0.6931471805599453f;
         }
     }
 
@@ -726,9 +813,9 @@ bool encode(CUtensorMap *map, const void *ptr, int64_t BH, int64_t L) {
 }  // namespace
 
 int launch_attn_sm100(const void *q, const void *k, const void *v, int64_t BH, int64_t Lq,
-                      int64_t Lk, float tau, const int32_t *kv_idx, const int32_t *kv_cnt,
-                      int64_t max_sel, void *out, float *lse, int32_t *status,
-                      cudaStream_t stream) {
+                           int64_t Lk, float tau, const int32_t *kv_idx, const int32_t *kv_cnt,
+                           int64_t max_sel, void *out, float *lse, int32_t *status,
+                           cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
     if (!encode(&mq, q, BH, Lq) || !encode(&mk, k, BH, Lk) || !encode(&mv, v, BH, Lk))
         return SPARSTAR_ECUDA;
@@ -736,9 +823,10 @@ int launch_attn_sm100(const void *q, const void *k, const void *v, int64_t BH, i
                              kSmemBytes) != cudaSuccess)
         return SPARSTAR_ECUDA;
     const int64_t nQB = ceil_div(Lq, kBlock), nKB = ceil_div(Lk, kBlock);
-    attn_sm100_kernel<<<(unsigned)(BH * nQB), kThreads, kSmemBytes, stream>>>(
-        mq, mk, mv, (int)Lq, (int)Lk, (int)nQB, (int)nKB, tau, kv_idx, kv_cnt, (int)max_sel,
-        static_cast<__nv_bfloat16 *>(out), lse, status);
+    const int64_t nPair = ceil_div(nQB, 2);
+    attn_sm100_kernel<<<(unsigned)(BH * nPair), kThreads, kSmemBytes, stream>>>(
+        mq, mk, mv, (int)Lq, (int)Lk, (int)nQB, (int)nKB, (int)nPair, tau, kv_idx, kv_cnt,
+        (int)max_sel, static_cast<__nv_bfloat16 *>(out), lse, status);
     return cudaGetLastError() == cudaSuccess ? SPARSTAR_OK : SPARSTAR_ECUDA;
 }
 

@@ -42,7 +42,8 @@ int64_t score_select_max_nkb(int D);
 int64_t score_select_tiled_max_nkb();
 int64_t score_select_ctas(int64_t BH, int64_t nQB);
 
-// Step 3, bf16 D=128: TMA + tcgen05 + TMEM kernel (sm_100a).
+// Step 3, bf16 D=128: TMA + tcgen05 + TMEM kernel (sm_100a), two query blocks
+// per CTA as interleaved pipelines.
 int launch_attn_sm100(const void *q, const void *k, const void *v, int64_t BH, int64_t Lq,
                       int64_t Lk, float tau, const int32_t *kv_idx, const int32_t *kv_cnt,
                       int64_t max_sel, void *out, float *lse, int32_t *status,
