@@ -103,3 +103,31 @@ def test_for_fp32_simt_bad_indices_flagged(sp, orc):
     idx = np.array([[[[0, 9], [2, 1]]]], np.int32)
     cnt = np.array([[[2, 2]]], np.int32)
     _run(sp, orc, w, idx=idx, cnt=cnt, expect_status=sp.STATUS_BAD_INDEX)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_uneven_list_lengths_within_pairs(sp, orc, seed):
+    """Query blocks run in pairs (2p, 2p+1), each with its own list: random
+    lengths from 0 to every key block (so the pairs see every mix of equal,
+    unequal, empty and longer-than-the-ring lists), random order, invalid
+    entries mixed in, an odd number of query blocks (the last pair has no
+    second block) and a partial last key block."""
+    rng = np.random.default_rng(seed)
+    w = synth.custom(H=2, D=128, dtype="bf16", text=256, ref=1900, cur=9 * 128 - 40,
+                     density=1.0, seed=40 + seed)
+    nQB, nKB = w.nQB, w.nKB
+    assert nQB % 2 == 1
+    max_sel = nKB + 4
+    idx = np.full((1, w.H, nQB, max_sel), -1, np.int32)
+    cnt = np.zeros((1, w.H, nQB), np.int32)
+    bad = False
+    for h in range(w.H):
+        for i in range(nQB):
+            n = int(rng.integers(0, nKB + 1))
+            lst = rng.permutation(nKB)[:n].tolist()
+            if n and rng.random() < 0.3:  # invalid entries are skipped
+                lst.insert(int(rng.integers(0, n)), int(rng.choice([-3, nKB, nKB + 9])))
+                bad = True
+            idx[0, h, i, :len(lst)] = lst
+            cnt[0, h, i] = len(lst)
+    _run(sp, orc, w, idx=idx, cnt=cnt, expect_status=sp.STATUS_BAD_INDEX if bad else 0)
