@@ -178,3 +178,24 @@ def test_fused_chain_in_a_cuda_graph(sp, orc, name):
         print(json.dumps({"workload": name, "graph_replay": True, "max_abs": max_abs,
                           "rel_l2": rel_l2}))
     del graph
+
+
+@pytest.mark.parametrize("dtype,D", [("f32", 64), ("f32", 128), ("bf16", 64)])
+def test_fused_chain_on_the_simt_attention_path(sp, orc, dtype, D):
+    """The three-launch chain where attention runs on the fp32 SIMT kernel
+    (fp32 inputs, or D = 64): lists bit-exact, outputs within tolerance."""
+    w = synth.custom(H=2, D=D, dtype=dtype, text=300, ref=700, cur=600, density=0.4, seed=21)
+    q, k, v = synth.generate(w)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse, ws = sp.sparstar_forward_fused(q.cuda(), k.cuda(), v.cuda(), w.text, w.image_ref,
+                                             w.ref, w.cur, w.density, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
+    _, _, _, idx32, cnt32 = orc.run_selection(qn, kn, w.text, w.image_ref, w.density)
+    assert np.array_equal(ws.kv_idx.cpu().numpy(), idx32)
+    assert np.array_equal(ws.kv_cnt.cpu().numpy(), cnt32)
+    rows = np.arange(w.B * w.H * w.Lq, dtype=np.int64)
+    want, want_lse = orc.attn_rows_f64(qn, kn, vn, idx32, cnt32, rows)
+    parity.check_out(parity.gather_rows(out, rows), want, w.dtype)
+    parity.check_lse(parity.gather_rows(lse, rows), want_lse, w.dtype)
