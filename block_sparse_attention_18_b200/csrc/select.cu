@@ -1,7 +1,7 @@
 // Step 2b — clip-aware block Top-K written straight into a forward-only
 // block list (SparSTAR, pith.science review, "What carries the argument":
 // text / Clip-1 reference blocks retained, reference and current blocks
-// ranked jointly under the density, only the forward mask fields written;
+// ranked jointly under the density, only the forward part of the mask kept;
 // "Referee Report", minor comment 5: block-wise Top-K).
 //
 // One warp per (b, h, query block) row.  Candidates are the blocks

@@ -10,8 +10,9 @@
  *
  * Sources (all on the pages describing SparSTAR, arXiv 2608.10519):
  *   [R-carry]  pith.science review of SparSTAR, "What carries the argument":
- *              contiguous 128-token blocks in attention-kernel order, block
- *              averaged q and k, S_ij = tau * qbar_i^T kbar_j with
+ *              contiguous 128-token blocks taken in the order the attention
+ *              kernel walks them, block-averaged q and k,
+ *              S_ij = tau * qbar_i^T kbar_j with
  *              tau = D^-1/2, the block-average identity, text (and, for
  *              Clip 1, the final image-pyramid reference) retained dense,
  *              reference and current blocks ranked jointly under a density
