@@ -661,7 +661,6 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             // m_ref = -inf only while every key so far was masked: then
             // every p is 0 (a finite offset keeps -inf * sc + offset = -inf).
             const float neg_m = m_ref > -INFINITY ? -m_ref : 0.0f;
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
             // P (bf16) in shared memory as the K-major, 128-byte-swizzled A
             // operand of O += P V: panel h holds keys 64h..64h+63, row r at
             // r * 128 bytes, 16-byte chunk c (keys 8c..8c+7) at c ^ (r & 7).
@@ -685,19 +684,24 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 prev_j = j - 1;
             }
             uint32_t pk[64];  // P of keys 2u, 2u+1 in pk[u]
+            // The exponent arguments come from the packed fp32x2 FMA (the
+            // same rounded fma per element as the scalar form, half the
+            // issues); the four running sums stay scalar adds.
+            const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(neg_m, neg_m);
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int u = 0; u < 64; u += 2) {
                 const int c = 2 * u;
-                const float p0 = ex2(fmaf(s[c], sc, neg_m));
-                const float p1 = ex2(fmaf(s[c + 1], sc, neg_m));
-                const float p2 = ex2(fmaf(s[c + 2], sc, neg_m));
-                const float p3 = ex2(fmaf(s[c + 3], sc, neg_m));
-                ls[0] += p0;
-                ls[1] += p1;
-                ls[2] += p2;
-                ls[3] += p3;
-                pk[u] = pack_bf16(p0, p1);
-                pk[u + 1] = pack_bf16(p2, p3);
+                const float2 x01 = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, nm2);
+                const float2 x23 = __ffma2_rn(make_float2(s[c + 2], s[c + 3]), sc2, nm2);
+                const float2 p01 = make_float2(ex2(x01.x), ex2(x01.y));
+                const float2 p23 = make_float2(ex2(x23.x), ex2(x23.y));
+                ls[0] += p01.x;
+                ls[1] += p01.y;
+                ls[2] += p23.x;
+                ls[3] += p23.y;
+                pk[u] = pack_bf16(p01.x, p01.y);
+                pk[u + 1] = pack_bf16(p23.x, p23.y);
             }
             l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             // Hand P over half by half: half h waits for the previous
