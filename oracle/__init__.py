@@ -18,7 +18,10 @@ attention over the selected blocks only.
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 (block-average identity, hand-derived order fixtures, brute-force top-k,
 dense-attention and masked-attention special cases against torch's
-scaled_dot_product_attention).  No function is parity unpinned.
+scaled_dot_product_attention), ``tests/test_oracle_mass_pins.py`` (retained
+mass) and ``tests/test_oracle_transfer_pins.py`` (lists carried across scales:
+identity, a 2x closed form, token-by-token brute force).  No function is
+parity unpinned.
 """
 import ctypes
 import os
@@ -56,6 +59,8 @@ def lib():
                                         vp, vp, i64, i64, vp, vp, vp]
         L.orc_retained_mass_f64.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i64,
                                             vp, vp, i64, i64, vp, vp, vp, vp, vp]
+        L.orc_transfer_lists.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64]
+        L.orc_transfer_lists.restype = i32
         _LIB = L
     return _LIB
 
@@ -204,6 +209,32 @@ def retained_mass_f64(q, k, kv_idx, kv_cnt, nF, rows):
                                 _ptr(out["lse_dense"]), _ptr(out["mass_block"]),
                                 _ptr(out["mass_tok"]), _ptr(out["mass_forced"]))
     return out
+
+
+def transfer_lists(kv_idx, kv_cnt, len_s, len_t, max_sel_t=None):
+    """Block lists of a source scale carried to a target scale by position
+    (the mask reuse the method argues against).  kv_idx [B,H,nQB_s,max_sel_s],
+    kv_cnt [B,H,nQB_s]; len_s, len_t: the four segment lengths (text,
+    image_ref, ref, cur) at each scale.  Returns (kv_idx_t, kv_cnt_t) with
+    max_sel_t = nKB_t unless given."""
+    kv_idx = np.ascontiguousarray(kv_idx, np.int32)
+    kv_cnt = np.ascontiguousarray(kv_cnt, np.int32)
+    B, H, _, max_sel_s = kv_idx.shape
+    ls = np.ascontiguousarray(len_s, np.int64)
+    lt = np.ascontiguousarray(len_t, np.int64)
+    assert ls.shape == (4,) and lt.shape == (4,)
+    assert kv_idx.shape[2] == nblocks(int(ls[3])) and kv_cnt.shape == kv_idx.shape[:3]
+    nKB_t = nblocks(int(lt.sum()))
+    nQB_t = nblocks(int(lt[3]))
+    if max_sel_t is None:
+        max_sel_t = nKB_t
+    idx_t = np.empty((B, H, nQB_t, max_sel_t), np.int32)
+    cnt_t = np.empty((B, H, nQB_t), np.int32)
+    rc = lib().orc_transfer_lists(_ptr(kv_idx), _ptr(kv_cnt), max_sel_s, B, H, _ptr(ls),
+                                  _ptr(lt), _ptr(idx_t), _ptr(cnt_t), max_sel_t)
+    if rc != 0:
+        raise ValueError("orc_transfer_lists: bad arguments (code %d)" % rc)
+    return idx_t, cnt_t
 
 
 def run_selection(q, k, text_len, image_ref_len, density):
