@@ -19,7 +19,8 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsparstar.so")
 
 SOURCES = ["sparstar_api.cu", "pool.cu", "score.cu", "select.cu", "score_select.cu",
-           "attn_simt.cu", "attn_sm100.cu", "forward_static.cu", "mass.cu"]
+           "attn_simt.cu", "attn_sm100.cu", "forward_static.cu", "mass.cu",
+           "transfer.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",

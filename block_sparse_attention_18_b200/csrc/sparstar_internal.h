@@ -65,4 +65,19 @@ cudaError_t launch_retained_mass(const void *q, const void *k, int dtype, int64_
                                  cudaStream_t stream);
 int64_t mass_max_nkb();
 
+// Diagnostic: block lists carried from a source scale to a target scale by
+// proportional token position (segments text, image_ref, ref, cur).
+struct TransferLayout {
+    int64_t len_s[4], len_t[4];  // segment lengths at the source and target scale
+    int64_t off_s[4], off_t[4];  // segment starts in the key sequence
+    int64_t Lk_t;                // keys at the target scale
+    int32_t nKB_s, nKB_t, nQB_s, nQB_t, nF_t;
+};
+TransferLayout make_transfer_layout(const int64_t *len_s, const int64_t *len_t);
+cudaError_t launch_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt,
+                                  int64_t src_max_sel, int64_t BH, const TransferLayout &ly,
+                                  int32_t *dst_idx, int32_t *dst_cnt, int64_t dst_max_sel,
+                                  cudaStream_t stream);
+int64_t transfer_max_nkb();
+
 }  // namespace sparstar

@@ -53,12 +53,14 @@ def _load():
                                          vp, vp, vp, vp, i64, vp, vp, vp, vp]
     L.sparstar_retained_mass.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, f32, i64, vp, vp,
                                          i64, vp, i64, vp, vp, vp, vp, vp, vp]
+    L.sparstar_transfer_lists.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp]
     L.sparstar_strerror.argtypes = [i32]
     L.sparstar_strerror.restype = ctypes.c_char_p
     L.sparstar_version.restype = i32
     for name in ("sparstar_block_pool", "sparstar_block_score", "sparstar_select",
                  "sparstar_attn_fwd", "sparstar_forward", "sparstar_block_pool_qk",
-                 "sparstar_score_select", "sparstar_forward_fused", "sparstar_retained_mass"):
+                 "sparstar_score_select", "sparstar_forward_fused", "sparstar_retained_mass",
+                 "sparstar_transfer_lists"):
         getattr(L, name).restype = i32
     return L
 
@@ -348,3 +350,28 @@ def sparstar_retained_mass(q, k, kv_idx, kv_cnt, n_forced_blocks: int, rows, tau
                                       _ptr(out["mass_tok"]), _ptr(out["mass_forced"]),
                                       _stream(stream)), "sparstar_retained_mass")
     return out
+
+
+def sparstar_transfer_lists(kv_idx, kv_cnt, src_len, dst_len, dst_idx=None, dst_cnt=None,
+                            stream=None):
+    """Diagnostic: block lists of a source scale carried by token position to
+    a target scale (mask reuse).  src_len / dst_len: the four segment lengths
+    (text, image_ref, ref, cur) at each scale.  Returns (dst_idx, dst_cnt)
+    with dst_max_sel = the target's key block count unless dst_idx is given."""
+    _dev(kv_idx, "kv_idx", torch.int32)
+    _dev(kv_cnt, "kv_cnt", torch.int32)
+    B, H = kv_idx.shape[0], kv_idx.shape[1]
+    ls = (ctypes.c_int64 * 4)(*[int(x) for x in src_len])
+    lt = (ctypes.c_int64 * 4)(*[int(x) for x in dst_len])
+    nKB_t = (sum(int(x) for x in dst_len) + BLOCK - 1) // BLOCK
+    nQB_t = (int(dst_len[3]) + BLOCK - 1) // BLOCK
+    if dst_idx is None:
+        dst_idx = torch.empty(B, H, nQB_t, nKB_t, device=kv_idx.device, dtype=torch.int32)
+    if dst_cnt is None:
+        dst_cnt = torch.empty(B, H, nQB_t, device=kv_idx.device, dtype=torch.int32)
+    _dev(dst_idx, "dst_idx", torch.int32)
+    _dev(dst_cnt, "dst_cnt", torch.int32)
+    _check(lib.sparstar_transfer_lists(_ptr(kv_idx), _ptr(kv_cnt), kv_idx.shape[-1], B, H, ls, lt,
+                                       _ptr(dst_idx), _ptr(dst_cnt), dst_idx.shape[-1],
+                                       _stream(stream)), "sparstar_transfer_lists")
+    return dst_idx, dst_cnt

@@ -313,6 +313,47 @@ int sparstar_retained_mass(const void *q, const void *k, int dtype, int64_t B, i
                            double *lse_dense, double *mass_block, double *mass_tok,
                            double *mass_forced, void *stream);
 
+/*
+ * sparstar_transfer_lists — diagnostic: the block lists of a source scale
+ * carried by token position to a target scale, i.e. the mask reuse across
+ * scales that the method argues against.  Source: pith.science review of
+ * SparSTAR, "Extended reading notes / Core claim" (reusing a block-selection
+ * pattern across scales loses retained attention mass, so the selection is
+ * recomputed at every scale) and Figure 1 (a reused support misses blocks
+ * that become active).  The pages give no map between two scales' token
+ * positions; this call implements the plainest one:
+ *   - keys at both scales are the segments [text | image_ref | ref | cur];
+ *     src_len[g] / dst_len[g] are their lengths at the source / target
+ *     scale (host arrays of 4 int64; queries are the cur segment);
+ *   - the target token at offset p of segment g maps to the source token at
+ *     offset floor(p * src_len[g] / dst_len[g]) of segment g (to none when
+ *     src_len[g] = 0);
+ *   - target query block i uses the list of the source query block holding
+ *     the image of its first query token, floor(128 i src_len[3] / dst_len[3]);
+ *   - target key block j is kept when j < ceil((dst_len[0] + dst_len[1]) /
+ *     128) (forced at the target), or when, for some segment g that j
+ *     overlaps, a listed source block meets the span [image of j's first
+ *     token in g, image of j's last token in g].
+ *   src_idx, src_cnt, src_max_sel: the source lists as written by
+ *            sparstar_select ([B,H,nQB_s,src_max_sel], [B,H,nQB_s] int32,
+ *            device); entries outside [0, nKB_s) are ignored and a count
+ *            above src_max_sel is read as src_max_sel
+ *   dst_idx  [B,H,nQB_t,dst_max_sel] int32 (device, written): kept blocks
+ *            ascending, unused slots -1
+ *   dst_cnt  [B,H,nQB_t] int32 (device, written)
+ * The transferred list has no budget of its own; dst_max_sel >= nKB_t (the
+ * target's key block count) always suffices and is required.
+ * Errors: SPARSTAR_EINVAL for null pointers, B or H < 1, a negative length,
+ * src_len[3] = 0 < dst_len[3], src_max_sel < 1 or more than 2^31 - 1
+ * source or target keys; SPARSTAR_ESIZE for dst_max_sel < nKB_t or a source
+ * with more than 32768 key blocks.  Nothing is launched on an error, or when
+ * dst_len[3] = 0 (no target rows).
+ */
+int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt, int64_t src_max_sel,
+                            int64_t B, int64_t H, const int64_t *src_len, const int64_t *dst_len,
+                            int32_t *dst_idx, int32_t *dst_cnt, int64_t dst_max_sel,
+                            void *stream);
+
 /* Message for a status code (static storage). */
 const char *sparstar_strerror(int code);
 

@@ -175,3 +175,26 @@ def test_retained_mass_argument_errors(sp):
     assert L.sparstar_retained_mass(*args(nF=-1)) == sp.EINVAL
     assert L.sparstar_retained_mass(*args(n=0)) == sp.EINVAL
     assert L.sparstar_retained_mass(*args(scratch=NUL)) == sp.EINVAL
+
+
+def test_transfer_lists_argument_errors(sp):
+    L = sp.lib
+    seg = lambda *v: (ctypes.c_int64 * 4)(*v)  # noqa: E731
+    src, dst = seg(128, 0, 256, 256), seg(128, 0, 512, 512)  # nKB_t = 9
+
+    def call(**kw):
+        return L.sparstar_transfer_lists(kw.get("idx", A), A, kw.get("src_max_sel", 4),
+                                         kw.get("B", 1), 1, kw.get("src", src),
+                                         kw.get("dst", dst), kw.get("out", A), A,
+                                         kw.get("dst_max_sel", 9), NUL)
+    assert call(idx=NUL) == sp.EINVAL
+    assert call(out=NUL) == sp.EINVAL
+    assert call(B=0) == sp.EINVAL
+    assert call(src_max_sel=0) == sp.EINVAL
+    assert call(src=NUL) == sp.EINVAL
+    assert call(src=seg(128, 0, -1, 256)) == sp.EINVAL
+    assert call(src=seg(128, 0, 256, 0)) == sp.EINVAL  # target queries without a source
+    assert call(dst_max_sel=8) == sp.ESIZE  # below nKB_t
+    assert call(src=seg(128, 0, 32768 * 128, 256)) == sp.ESIZE  # source bitmap limit
+    # no target rows: nothing to do, nothing launched, even without a device
+    assert call(dst=seg(128, 0, 512, 0), dst_max_sel=5) == sp.OK

@@ -47,8 +47,13 @@ def _run(sp, orc, w, rows, q=None, k=None, v=None):
                                     torch.from_numpy(rows).cuda())
     torch.cuda.synchronize()
     got = {n: t.cpu().numpy() for n, t in got.items()}
-    want = orc.retained_mass_f64(qn, kn, ws.kv_idx.cpu().numpy(), ws.kv_cnt.cpu().numpy(),
-                                 ws.n_forced, rows)
+    # The oracle gets its own lists (its fp32 selection), which the GPU's
+    # lists must equal bit for bit; no oracle input comes from the GPU.
+    _, _, _, oidx, ocnt = orc.run_selection(qn, kn, w.text, w.image_ref, w.density)
+    gidx, sel = ws.kv_idx.cpu().numpy(), oidx.shape[-1]
+    assert np.array_equal(gidx[..., :sel], oidx) and (gidx[..., sel:] == -1).all()
+    assert np.array_equal(ws.kv_cnt.cpu().numpy(), ocnt)
+    want = orc.retained_mass_f64(qn, kn, oidx, ocnt, ws.n_forced, rows)
     for n in ("mass_block", "mass_tok", "mass_forced"):
         err = float(np.max(np.abs(got[n] - want[n])))
         assert err <= MASS_TOL, "%s: max err %.3g" % (n, err)
