@@ -321,19 +321,21 @@ int sparstar_retained_mass(const void *q, const void *k, int dtype, int64_t B, i
  * pattern across scales loses retained attention mass, so the selection is
  * recomputed at every scale) and Figure 1 (a reused support misses blocks
  * that become active).  The pages give no map between two scales' token
- * positions; this call implements the plainest one:
+ * positions; this call resamples the block mask by nearest neighbour
+ * along the token order, the plainest reading:
  *   - keys at both scales are the segments [text | image_ref | ref | cur];
  *     src_len[g] / dst_len[g] are their lengths at the source / target
  *     scale (host arrays of 4 int64; queries are the cur segment);
- *   - the target token at offset p of segment g maps to the source token at
- *     offset floor(p * src_len[g] / dst_len[g]) of segment g (to none when
- *     src_len[g] = 0);
+ *   - the target token at offset p of segment g has as image the source
+ *     token at offset floor(p * src_len[g] / dst_len[g]) of segment g (none
+ *     when src_len[g] = 0);
+ *   - the centre of a block of n real tokens starting at token a is token
+ *     a + (n - 1) / 2;
  *   - target query block i uses the list of the source query block holding
- *     the image of its first query token, floor(128 i src_len[3] / dst_len[3]);
+ *     the image of i's centre query token;
  *   - target key block j is kept when j < ceil((dst_len[0] + dst_len[1]) /
- *     128) (forced at the target), or when, for some segment g that j
- *     overlaps, a listed source block meets the span [image of j's first
- *     token in g, image of j's last token in g].
+ *     128) (forced at the target), or when the image of j's centre token
+ *     lies in a block of that list.
  *   src_idx, src_cnt, src_max_sel: the source lists as written by
  *            sparstar_select ([B,H,nQB_s,src_max_sel], [B,H,nQB_s] int32,
  *            device); entries outside [0, nKB_s) are ignored and a count
@@ -341,8 +343,9 @@ int sparstar_retained_mass(const void *q, const void *k, int dtype, int64_t B, i
  *   dst_idx  [B,H,nQB_t,dst_max_sel] int32 (device, written): kept blocks
  *            ascending, unused slots -1
  *   dst_cnt  [B,H,nQB_t] int32 (device, written)
- * The transferred list has no budget of its own; dst_max_sel >= nKB_t (the
- * target's key block count) always suffices and is required.
+ * The transferred list has no budget of its own (it keeps about the source
+ * scale's density); dst_max_sel >= nKB_t (the target's key block count)
+ * always suffices and is required.
  * Errors: SPARSTAR_EINVAL for null pointers, B or H < 1, a negative length,
  * src_len[3] = 0 < dst_len[3], src_max_sel < 1 or more than 2^31 - 1
  * source or target keys; SPARSTAR_ESIZE for dst_max_sel < nKB_t or a source

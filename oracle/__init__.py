@@ -20,7 +20,7 @@ Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 dense-attention and masked-attention special cases against torch's
 scaled_dot_product_attention), ``tests/test_oracle_mass_pins.py`` (retained
 mass) and ``tests/test_oracle_transfer_pins.py`` (lists carried across scales:
-identity, a 2x closed form, token-by-token brute force).  No function is
+identity, a 2x closed form, the inverse formulation).  No function is
 parity unpinned.
 """
 import ctypes

@@ -543,26 +543,41 @@ void orc_retained_mass_f64(const void *q, const void *k, int dtype, int64_t B, i
 
 /* --------------------------------------- diagnostic: lists reused across scales */
 
+/* The image of one target token: its segment g's source token at offset
+ * floor(p * len_s[g] / len_t[g]), or -1 when len_s[g] = 0. */
+static int64_t orc_image(int64_t t, const int64_t *off_s, const int64_t *off_t,
+                         const int64_t *len_s, const int64_t *len_t)
+{
+    for (int g = 0; g < 4; ++g) {
+        if (t >= off_t[g] && t < off_t[g] + len_t[g]) {
+            if (len_s[g] == 0) return -1;
+            return off_s[g] + (t - off_t[g]) * len_s[g] / len_t[g];
+        }
+    }
+    return -1;
+}
+
 /* The block lists of a source scale carried to a target scale by position:
  * the "reuse" that the method argues against ([R-core]: reusing a
  * block-selection pattern across scales loses retained attention mass, so
  * the selection is recomputed at every scale; the review's Figure 1: a
  * reused support misses blocks that become active at the new scale).  The
  * pages give no map between two scales' token positions; the reading used
- * (listed in the design notes):
+ * (listed in the design notes) resamples the block mask by nearest
+ * neighbour along the token order:
  *   - keys at both scales are the segments [text | image_ref | ref | cur];
  *     segment g has len_s[g] tokens at the source and len_t[g] at the
  *     target (queries are the cur segment);
- *   - the target token at offset p of segment g maps to the source token at
- *     offset floor(p * len_s[g] / len_t[g]) of the same segment, and to none
- *     when len_s[g] = 0;
- *   - target query block i uses the list of the source query block that
- *     holds the image of its first query token;
- *   - target key block j is kept when j < nF_t (forced at the target scale)
- *     or when, for some segment g that j overlaps, a source block that
- *     meets the span [image of j's first token in g, image of j's last
- *     token in g] is in that list.  For ratios len_s / len_t up to 128 this
- *     is the same as asking whether any token of j maps into a listed block.
+ *   - the target token at offset p of segment g has as image the source
+ *     token at offset floor(p * len_s[g] / len_t[g]) of the same segment,
+ *     and none when len_s[g] = 0;
+ *   - the centre of a block of n real tokens starting at token a is token
+ *     a + floor((n - 1) / 2);
+ *   - target query block i uses the list of the source query block holding
+ *     the image of i's centre query token;
+ *   - target key block j is kept when j < nF_t (forced at the target) or
+ *     when the source block holding the image of j's centre token is in
+ *     that list.
  * Output kv_idx_t [B,H,nQB_t,max_sel_t]: the kept blocks ascending, unused
  * slots -1; kv_cnt_t [B,H,nQB_t].  Source entries outside [0, nKB_s) are
  * ignored; a source count above max_sel_s is read as max_sel_s.
@@ -587,9 +602,11 @@ int orc_transfer_lists(const int32_t *idx_s, const int32_t *cnt_s, int64_t max_s
     for (int64_t row = 0; row < B * H * nQB_t; ++row) {
         const int64_t bh = row / nQB_t;
         const int64_t i = row % nQB_t;
-        /* the source row: the block of the image of query token 128 i */
-        const int64_t src_q = (i * ORC_BLOCK) * len_s[3] / len_t[3];
-        const int64_t src_row = bh * nQB_s + src_q / ORC_BLOCK;
+        /* the source row: the block of the image of i's centre query token */
+        const int64_t qa = i * ORC_BLOCK;
+        const int64_t qn = (len_t[3] - qa < ORC_BLOCK) ? len_t[3] - qa : ORC_BLOCK;
+        const int64_t q_img = (qa + (qn - 1) / 2) * len_s[3] / len_t[3];
+        const int64_t src_row = bh * nQB_s + q_img / ORC_BLOCK;
         int64_t n_src = cnt_s[src_row];
         if (n_src > max_sel_s) n_src = max_sel_s;
         if (n_src < 0) n_src = 0;
@@ -597,21 +614,18 @@ int orc_transfer_lists(const int32_t *idx_s, const int32_t *cnt_s, int64_t max_s
         int64_t n = 0;
         for (int64_t j = 0; j < nKB_t; ++j) {
             int keep = j < nF_t;
-            const int64_t a = j * ORC_BLOCK;
-            const int64_t b = (a + ORC_BLOCK - 1 < Lk_t - 1) ? a + ORC_BLOCK - 1 : Lk_t - 1;
-            for (int g = 0; g < 4 && !keep; ++g) {
-                const int64_t lo = a > off_t[g] ? a : off_t[g];
-                const int64_t end = off_t[g] + len_t[g] - 1;
-                const int64_t hi = b < end ? b : end;
-                if (lo > hi || len_s[g] == 0) continue;
-                const int64_t ps = off_s[g] + (lo - off_t[g]) * len_s[g] / len_t[g];
-                const int64_t pe = off_s[g] + (hi - off_t[g]) * len_s[g] / len_t[g];
-                for (int64_t sb = ps / ORC_BLOCK; sb <= pe / ORC_BLOCK && !keep; ++sb)
+            if (!keep) {
+                const int64_t a = j * ORC_BLOCK;
+                const int64_t nj = (Lk_t - a < ORC_BLOCK) ? Lk_t - a : ORC_BLOCK;
+                const int64_t img = orc_image(a + (nj - 1) / 2, off_s, off_t, len_s, len_t);
+                if (img >= 0) {
+                    const int64_t sb = img / ORC_BLOCK;
                     for (int64_t c = 0; c < n_src; ++c)
                         if (list[c] >= 0 && list[c] < nKB_s && list[c] == sb) {
                             keep = 1;
                             break;
                         }
+                }
             }
             if (keep) idx_t[row * max_sel_t + n++] = (int32_t)j;
         }

@@ -5,18 +5,24 @@ claim" (reusing a block-selection pattern across scales loses retained
 attention mass; the method recomputes the selection at every scale) and
 Figure 1 (a reused support misses blocks that become active).  The pages give
 no map between the token positions of two scales.  The reading pinned here
-maps each key segment (text, image_ref, ref, cur) proportionally along its
-token order: target offset p of segment g maps to source offset
-floor(p * len_s[g] / len_t[g]).  Target query block i takes the list of the
-source block that holds the image of its first query token.  A target key
-block is kept when it is forced at the target, or when its image meets a
-listed source block.
+resamples the block mask by nearest neighbour along each key segment (text,
+image_ref, ref, cur):
+- target offset p of segment g has as image the source offset
+  floor(p * len_s[g] / len_t[g]);
+- a block's centre is its token a + (n - 1) // 2;
+- target query block i reads the list of the source block that holds the
+  image of its centre query token;
+- target key block j is kept when it is forced at the target, or when the
+  image of its centre token lies in a listed source block.
 
 Each test checks the oracle against something other than its own code:
 - the identity map (the list comes back with the target's forced prefix);
 - an exact 2x refinement with a closed form;
-- a token-by-token brute force in plain Python on random small layouts
-  (the oracle works on spans; the two agree while len_s / len_t <= 128);
+- the inverse formulation in plain Python on random ragged layouts: for
+  every listed source block, the target offsets whose image falls in it form
+  the integer interval [ceil(lo * lt / ls), ceil((hi + 1) * lt / ls) - 1],
+  and the target blocks whose centre lies in one of those intervals are kept;
+- single-block lists at every source block;
 - the invariants of a valid list;
 - the error returns.
 """
@@ -46,42 +52,55 @@ def _random_lists(rng, B, H, nQB, nKB, max_sel, p_invalid=0.0):
     return idx, cnt
 
 
-def _brute(idx_s, cnt_s, len_s, len_t):
-    """Token by token: keep target block j if it is forced at the target or
-    if any of its tokens maps into a source block the source row lists."""
+def _cdiv(a, b):
+    return -(-a // b)
+
+
+def _inverse(idx_s, cnt_s, len_s, len_t):
+    """From the source side: the target blocks whose centre lies in the
+    preimage of a listed source block (and the forced prefix)."""
     B, H, nQB_s, max_sel_s = idx_s.shape
-    off_s = np.concatenate([[0], np.cumsum(len_s)[:-1]])
-    off_t = np.concatenate([[0], np.cumsum(len_t)[:-1]])
+    off_s = [int(x) for x in np.concatenate([[0], np.cumsum(len_s)[:-1]])]
+    off_t = [int(x) for x in np.concatenate([[0], np.cumsum(len_t)[:-1]])]
     Lk_s, Lk_t = int(sum(len_s)), int(sum(len_t))
     nKB_s, nKB_t = _nb(Lk_s), _nb(Lk_t)
     nQB_t = _nb(len_t[3])
     nF_t = _nb(len_t[0] + len_t[1])
-    # segment and offset of every target token
-    seg_t = np.zeros(Lk_t, np.int64)
-    for g in range(4):
-        seg_t[off_t[g]:off_t[g] + len_t[g]] = g
+    ls_c, lt_c = int(len_s[3]), int(len_t[3])
+
+    def centre(a, L):
+        return a + (min(BLOCK, L - a) - 1) // 2
+
+    # query side: source query block s covers target query offsets
+    # [ceil(128 s lt / ls), ceil(128 (s+1) lt / ls) - 1]
+    q_src = {}
+    for i in range(nQB_t):
+        c = centre(i * BLOCK, lt_c)
+        for sblk in range(nQB_s):
+            lo = _cdiv(sblk * BLOCK * lt_c, ls_c)
+            hi = _cdiv(min((sblk + 1) * BLOCK, ls_c) * lt_c, ls_c) - 1
+            if lo <= c <= hi:
+                q_src[i] = sblk
     out = {}
     for b in range(B):
         for h in range(H):
             for i in range(nQB_t):
-                src_q = (i * BLOCK) * len_s[3] // len_t[3]
-                si = src_q // BLOCK
+                si = q_src[i]
                 n = min(int(cnt_s[b, h, si]), max_sel_s)
                 listed = {int(x) for x in idx_s[b, h, si, :max(n, 0)] if 0 <= x < nKB_s}
-                kept = []
-                for j in range(nKB_t):
-                    keep = j < nF_t
-                    for t in range(j * BLOCK, min((j + 1) * BLOCK, Lk_t)):
-                        if keep:
-                            break
-                        g = int(seg_t[t])
-                        if len_s[g] == 0:
+                kept = set(range(nF_t))
+                for sb in listed:
+                    for g in range(4):
+                        lo = max(sb * BLOCK, off_s[g]) - off_s[g]
+                        hi = min(sb * BLOCK + BLOCK, off_s[g] + len_s[g]) - 1 - off_s[g]
+                        if lo > hi or len_t[g] == 0:
                             continue
-                        src_tok = off_s[g] + (t - off_t[g]) * len_s[g] // len_t[g]
-                        keep = (src_tok // BLOCK) in listed
-                    if keep:
-                        kept.append(j)
-                out[(b, h, i)] = kept
+                        t_lo = off_t[g] + _cdiv(lo * len_t[g], len_s[g])
+                        t_hi = off_t[g] + _cdiv((hi + 1) * len_t[g], len_s[g]) - 1
+                        for j in range(nKB_t):
+                            if t_lo <= centre(j * BLOCK, Lk_t) <= t_hi:
+                                kept.add(j)
+                out[(b, h, i)] = sorted(kept)
     return out
 
 
@@ -124,7 +143,7 @@ def test_exact_2x_refinement_closed_form(orc):
 
 
 @pytest.mark.parametrize("seed", range(16))
-def test_matches_token_brute_force_on_random_layouts(orc, seed):
+def test_matches_the_inverse_formulation_on_random_layouts(orc, seed):
     rng = np.random.default_rng(100 + seed)
     text = int(rng.integers(1, 300))
     img = int(rng.choice([0, int(rng.integers(1, 400))]))
@@ -136,20 +155,21 @@ def test_matches_token_brute_force_on_random_layouts(orc, seed):
     len_s, len_t = [text, img, ref_s, cur_s], [text, img, ref_t, cur_t]
     nKB_s, nQB_s = _nb(sum(len_s)), _nb(cur_s)
     idx, cnt = _random_lists(rng, 1, 2, nQB_s, nKB_s, max(1, nKB_s // 2), p_invalid=0.1)
-    expect = _brute(idx, cnt, len_s, len_t)
+    expect = _inverse(idx, cnt, len_s, len_t)
     _check_against(orc.transfer_lists(idx, cnt, len_s, len_t), expect)
 
 
 def test_segment_absent_at_the_source_maps_to_nothing(orc):
-    # The reference segment is empty at the source: target reference blocks
-    # can only be kept through a straddling piece of another segment.
+    # The reference segment is empty at the source: a target block whose
+    # centre is a reference token has no image and is never kept.
     len_s, len_t = [128, 0, 0, 512], [128, 0, 640, 512]
     nKB_s = _nb(sum(len_s))
     idx = np.tile(np.arange(nKB_s, dtype=np.int32), (1, 1, _nb(512), 1))
     cnt = np.full((1, 1, _nb(512)), nKB_s, np.int32)
-    expect = _brute(idx, cnt, len_s, len_t)
+    expect = _inverse(idx, cnt, len_s, len_t)
     _check_against(orc.transfer_lists(idx, cnt, len_s, len_t), expect)
     idx_t, cnt_t = orc.transfer_lists(idx, cnt, len_s, len_t)
+    # target blocks 1..5 hold reference tokens only
     assert all(j not in range(1, 6) for j in idx_t[0, 0, 0, :cnt_t[0, 0, 0]])
 
 
@@ -183,9 +203,8 @@ def test_error_returns(orc):
     ([100, 0, 700, 500], [100, 0, 420, 300]),
     ([100, 0, 252, 180], [100, 0, 420, 300]),
     ([100, 0, 735, 525], [100, 0, 420, 300]),
-    # here the last token of one target block is the only one whose image
-    # falls in the next source block
     ([100, 0, 559, 495], [100, 0, 435, 385]),
+    ([1, 0, 127, 129], [1, 0, 1000, 1001]),
 ])
 def test_single_block_lists_at_every_source_block(orc, layout):
     # Each source row lists one block; over the heads every source block is
@@ -198,5 +217,5 @@ def test_single_block_lists_at_every_source_block(orc, layout):
         for i in range(nQB_s):
             idx[0, h, i, 0] = (h + 3 * i) % nKB_s
     cnt = np.ones((1, H, nQB_s), np.int32)
-    expect = _brute(idx, cnt, len_s, len_t)
+    expect = _inverse(idx, cnt, len_s, len_t)
     _check_against(orc.transfer_lists(idx, cnt, len_s, len_t), expect)
