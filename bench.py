@@ -461,6 +461,11 @@ def run_gpu(args, world, rank, local):
 
     dense = dense_comparison(sp, w, qd, kd, vd, tau, per["attn"], stream) if args.dense else None
     mass = retained_mass(sp, w, qd, kd, ws, lse, args.mass_rows) if args.mass_rows > 0 else None
+    reuse = None
+    if args.reuse and args.mass_rows > 0:
+        front_ms = sum(t for n, t in per.items() if n != "attn")
+        reuse = reuse_across_scales(sp, w, qd, kd, vd, tau, ws.n_forced, per["attn"], front_ms,
+                                    args.mass_rows, stream)
 
     if rank != 0:
         return
@@ -497,10 +502,89 @@ def run_gpu(args, world, rank, local):
         line["dense_comparison"] = dense
     if mass is not None:
         line["retained_mass"] = mass
+    if reuse is not None:
+        line["reuse_across_scales"] = reuse
     if world == 1 and not args.no_cpu_baseline:
         qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
         line["cpu_baseline"] = cpu_baseline(w, qn, kn, vn, flops)
     print(json.dumps(line), flush=True)
+
+
+def mass_rows(w, per_head, device, seed=0):
+    """Per head: the first row, the last row and `per_head` seeded random
+    query rows, as flat row indices (bh * Lq + r)."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for bh in range(w.B * w.H):
+        r = {0, w.Lq - 1, *rng.choice(w.Lq, per_head, replace=False).tolist()}
+        rows.extend(bh * w.Lq + x for x in sorted(r))
+    return torch.tensor(rows, dtype=torch.int64, device=device)
+
+
+def reuse_across_scales(sp, w, qd, kd, vd, tau, n_forced, fresh_attn_ms, fresh_front_ms,
+                        per_head, stream, reps=5):
+    """Diagnostic, outside the timed region: the block lists selected at the
+    previous scale of the schedule, carried to this scale by position
+    (sparstar_transfer_lists), as a replacement for this scale's fresh
+    selection.  The source-scale inputs are either an independent seeded
+    draw of that scale's workload (no persistence of content between the
+    scales) or this scale's own tokens taken at the source positions (full
+    persistence under the same position map); the two bracket what real
+    activations would give.  For each: the transfer's time and bytes, the
+    attention's time over the reused lists, their density and the retained
+    attention mass on the sampled rows, beside the fresh lists' mass."""
+    prev = synth.PREVIOUS_SCALE.get(w.name)
+    if prev is None:
+        return None
+    src = synth.WORKLOADS[prev]
+    seg_s, seg_t = synth.segments(src), synth.segments(w)
+    nF_s = sp.sparstar_forced_blocks(src.text, src.image_ref)
+    rows_t = mass_rows(w, per_head, qd.device)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    qs, ks, _ = synth.generate(src)
+    sources = {"independent": (qs.cuda(), ks.cuda())}
+    del qs, ks
+    sources["subsampled"] = synth.coarser_scale(qd, kd, seg_t, seg_s)
+    out = {"source_scale": prev, "source_density": src.density, "target_density": w.density,
+           "map": "per-segment proportional token position (text, image_ref, ref, cur)",
+           "fresh_front_end_ms": fresh_front_ms, "fresh_attn_ms": fresh_attn_ms}
+    o = torch.empty_like(qd)
+    for name, (a, b) in sources.items():
+        qbar, kbar = sp.sparstar_block_pool_qk(a, b, stream=stream)
+        sidx, scnt = sp.sparstar_score_select(qbar, kbar, nF_s, src.density, stream=stream)
+        tidx, tcnt = sp.sparstar_transfer_lists(sidx, scnt, seg_s, seg_t, stream=stream)
+        t_ms = timed(lambda: sp.sparstar_transfer_lists(sidx, scnt, seg_s, seg_t, tidx, tcnt,
+                                                        stream=stream))
+        a_ms = timed(lambda: sp.sparstar_attn_fwd(qd, kd, vd, tidx, tcnt, tau, o, None,
+                                                  want_lse=False, stream=stream))
+        m = sp.sparstar_retained_mass(qd, kd, tidx, tcnt, n_forced, rows_t)
+        torch.cuda.synchronize()
+        cnt = tcnt.double()
+        moved = 4 * (sidx.numel() + scnt.numel() + tidx.numel() + tcnt.numel())
+        out[name] = {
+            "transfer_ms": t_ms, "transfer_bytes": moved,
+            "transfer_gbs": moved / (t_ms * 1e-3) / 1e9,
+            "attn_ms": a_ms,
+            "attn_tflops": attention_flops(tidx.cpu().numpy(), tcnt.cpu().numpy(), w.Lq, w.Lk,
+                                           w.D) / (a_ms * 1e-3) / 1e12,
+            "mean_blocks_per_row": float(cnt.mean()),
+            "density_of_candidates": float(((cnt - n_forced) / (w.nKB - n_forced)).mean()),
+            "mass_block_mean": float(m["mass_block"].mean()),
+            "mass_tok_mean": float(m["mass_tok"].mean()),
+        }
+        del qbar, kbar, sidx, scnt, tidx, tcnt
+    return out
 
 
 def retained_mass(sp, w, qd, kd, ws, lse, per_head, seed=0):
@@ -510,12 +594,8 @@ def retained_mass(sp, w, qd, kd, ws, lse, per_head, seed=0):
     the token-wise bound (the same forced blocks plus the M largest candidate
     weights, M = the lists' candidate tokens).  Also checks that the block
     mass equals exp(lse_sparse - lse_dense) with the attention kernel's LSE."""
-    rng = np.random.default_rng(seed)
-    rows = []
-    for bh in range(w.B * w.H):
-        r = {0, w.Lq - 1, *rng.choice(w.Lq, per_head, replace=False).tolist()}
-        rows.extend(bh * w.Lq + x for x in sorted(r))
-    rows_t = torch.tensor(rows, dtype=torch.int64, device=qd.device)
+    rows_t = mass_rows(w, per_head, qd.device, seed)
+    rows = rows_t.tolist()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     got = sp.sparstar_retained_mass(qd, kd, ws.kv_idx, ws.kv_cnt, ws.n_forced, rows_t)
@@ -584,6 +664,9 @@ def main(argv=None):
     ap.add_argument("--mass-rows", type=int, default=64,
                     help="random query rows per head for the retained-mass diagnostic "
                          "(0 skips it)")
+    ap.add_argument("--no-reuse", dest="reuse", action="store_false",
+                    help="skip the mask-reuse diagnostic (lists of the previous scale carried "
+                         "to this one)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense comparison point (density 1 and torch SDPA)")

@@ -5,21 +5,20 @@
 // is why the method recomputes the selection at every scale; Figure 1 of the
 // review: a reused support misses blocks that become active).
 //
-// The pages give no map between two scales' token positions.  Reading: each
-// key segment g of [text | image_ref | ref | cur] maps proportionally along
-// its token order, target offset p -> source offset floor(p * len_s[g] /
-// len_t[g]) (none when len_s[g] = 0).  Target query block i takes the list of
-// the source query block that holds the image of its first query token.
-// Target key block j is kept when j < nF_t, or when for some segment g that
-// j overlaps a listed source block meets [image of j's first token in g,
-// image of j's last token in g].
+// The pages give no map between two scales' token positions.  Reading: the
+// block mask is resampled by nearest neighbour along each key segment g of
+// [text | image_ref | ref | cur]: target offset p has as image the source
+// offset floor(p * len_s[g] / len_t[g]) (none when len_s[g] = 0).  Target
+// query block i takes the list of the source query block that holds the
+// image of i's centre query token; target key block j is kept when j < nF_t
+// or when the image of j's centre token lies in a listed source block (the
+// centre of a block of n real tokens starting at a is a + (n - 1) / 2).
 //
 // One warp per target row, eight rows in flight per CTA:
 //   1. the source row's list becomes a bitmap in shared memory (one bit per
 //      source key block, entries outside [0, nKB_s) dropped);
 //   2. the 32 lanes test 32 consecutive target blocks at a time: each lane
-//      maps the (at most four) segment pieces of its block to source block
-//      ranges and looks them up in the bitmap;
+//      maps its block's centre token to the source and looks up the bit;
 //   3. a ballot and a prefix popcount write the kept blocks in ascending
 //      order; the rest of the row is filled with -1.
 // Memory: the source lists are read once and the target lists written once
@@ -44,9 +43,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
          row += (int64_t)gridDim.x * kWarpsPerCta) {
         const int64_t bh = row / ly.nQB_t;
         const int64_t i = row % ly.nQB_t;
-        // the source row: the block of the image of query token 128 i
-        const int64_t src_q = (i * kBlock) * ly.len_s[3] / ly.len_t[3];
-        const int64_t src_row = bh * ly.nQB_s + src_q / kBlock;
+        // the source row: the block of the image of i's centre query token
+        const int64_t qa = i * kBlock;
+        const int64_t qn = ly.len_t[3] - qa < kBlock ? ly.len_t[3] - qa : kBlock;
+        const int64_t q_img = (qa + (qn - 1) / 2) * ly.len_s[3] / ly.len_t[3];
+        const int64_t src_row = bh * ly.nQB_s + q_img / kBlock;
 
         for (int w = lane; w < words; w += 32) bm[w] = 0u;
         __syncwarp();
@@ -66,19 +67,18 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
             bool keep = false;
             if (j < ly.nKB_t) {
                 keep = j < ly.nF_t;
-                const int64_t a = (int64_t)j * kBlock;
-                const int64_t b = a + kBlock - 1 < ly.Lk_t - 1 ? a + kBlock - 1 : ly.Lk_t - 1;
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int64_t lo = a > ly.off_t[g] ? a : ly.off_t[g];
-                    const int64_t end = ly.off_t[g] + ly.len_t[g] - 1;
-                    const int64_t hi = b < end ? b : end;
-                    if (keep || lo > hi || ly.len_s[g] == 0) continue;
-                    // images of the piece's first and last token (< len_s[g])
-                    const int64_t ps = ly.off_s[g] + (lo - ly.off_t[g]) * ly.len_s[g] / ly.len_t[g];
-                    const int64_t pe = ly.off_s[g] + (hi - ly.off_t[g]) * ly.len_s[g] / ly.len_t[g];
-                    for (int64_t sb = ps / kBlock; sb <= pe / kBlock && !keep; ++sb)
+                if (!keep) {
+                    const int64_t a = (int64_t)j * kBlock;
+                    const int64_t n_real = ly.Lk_t - a < kBlock ? ly.Lk_t - a : kBlock;
+                    const int64_t t = a + (n_real - 1) / 2;  // the block's centre token
+                    int g = 0;
+                    while (g < 3 && t >= ly.off_t[g] + ly.len_t[g]) ++g;
+                    if (ly.len_s[g] > 0) {
+                        const int64_t img =
+                            ly.off_s[g] + (t - ly.off_t[g]) * ly.len_s[g] / ly.len_t[g];
+                        const int64_t sb = img / kBlock;
                         keep = (bm[sb >> 5] >> (sb & 31)) & 1u;
+                    }
                 }
             }
             const uint32_t ballot = __ballot_sync(0xffffffffu, keep);

@@ -142,3 +142,43 @@ def as_numpy(t: torch.Tensor):
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view("uint16")
     return t.numpy()
+
+
+# The scale before each scale of the sweep schedule (same clip layout), used
+# by the mask-reuse diagnostic; `largest` has the Clip 2+ layout of the 72k
+# scale.
+PREVIOUS_SCALE = {
+    "largest": "sweep_clip2_40500",
+    **{"sweep_%s_%d" % (tag, b): "sweep_%s_%d" % (tag, a)
+       for tag in ("clip1", "clip2")
+       for a, b in ((8000, 18000), (18000, 40500), (40500, 72000))},
+}
+
+
+def segments(w: Workload):
+    """Key segment lengths (text, image_ref, ref, cur); queries are cur."""
+    return [w.text, w.image_ref, w.ref, w.cur]
+
+
+def coarser_scale(q: torch.Tensor, k: torch.Tensor, seg_t, seg_s):
+    """Source-scale inputs that carry the target scale's content: source
+    offset p of segment g takes the target token at offset
+    floor(p * len_t[g] / len_s[g]) of that segment (the same proportional
+    position map as the cross-scale list transfer).  q is the cur segment.
+    Works on any device; returns (q_s, k_s)."""
+    dev = q.device
+
+    def pick(len_t, len_s, start):
+        p = torch.arange(len_s, device=dev, dtype=torch.int64)
+        return start + (p * len_t) // len_s
+
+    q_idx = pick(seg_t[3], seg_s[3], 0)
+    k_parts, off = [], 0
+    for g in range(4):
+        if seg_s[g] > 0:
+            if seg_t[g] == 0:
+                raise ValueError("segment %d exists at the source but not at the target" % g)
+            k_parts.append(pick(seg_t[g], seg_s[g], off))
+        off += seg_t[g]
+    k_idx = torch.cat(k_parts)
+    return q.index_select(2, q_idx).contiguous(), k.index_select(2, k_idx).contiguous()
