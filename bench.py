@@ -552,6 +552,29 @@ def reuse_across_scales(sp, w, qd, kd, vd, tau, n_forced, fresh_attn_ms, fresh_f
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / reps
 
+    def timed_graph(fn):
+        # A short kernel: launched eagerly its time is the host's launch
+        # overhead, so the repetitions are replayed from a CUDA graph.
+        # fn(st) launches on stream st.
+        fn(stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap), torch.cuda.graph(g, stream=cap):
+            for _ in range(reps):
+                fn(cap)
+        stream.wait_stream(cap)
+        with torch.cuda.stream(stream):
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
     qs, ks, _ = synth.generate(src)
     sources = {"independent": (qs.cuda(), ks.cuda())}
     del qs, ks
@@ -564,8 +587,8 @@ def reuse_across_scales(sp, w, qd, kd, vd, tau, n_forced, fresh_attn_ms, fresh_f
         qbar, kbar = sp.sparstar_block_pool_qk(a, b, stream=stream)
         sidx, scnt = sp.sparstar_score_select(qbar, kbar, nF_s, src.density, stream=stream)
         tidx, tcnt = sp.sparstar_transfer_lists(sidx, scnt, seg_s, seg_t, stream=stream)
-        t_ms = timed(lambda: sp.sparstar_transfer_lists(sidx, scnt, seg_s, seg_t, tidx, tcnt,
-                                                        stream=stream))
+        t_ms = timed_graph(lambda st: sp.sparstar_transfer_lists(sidx, scnt, seg_s, seg_t, tidx,
+                                                                 tcnt, stream=st))
         a_ms = timed(lambda: sp.sparstar_attn_fwd(qd, kd, vd, tidx, tcnt, tau, o, None,
                                                   want_lse=False, stream=stream))
         m = sp.sparstar_retained_mass(qd, kd, tidx, tcnt, n_forced, rows_t)

@@ -269,13 +269,12 @@ SPARSTAR_API int sparstar_retained_mass(const void *q, const void *k, int dtype,
         static_cast<cudaStream_t>(stream)));
 }
 
-SPARSTAR_API int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt,
-                                         int64_t src_max_sel, int64_t B, int64_t H,
-                                         const int64_t *src_len, const int64_t *dst_len,
-                                         int32_t *dst_idx, int32_t *dst_cnt, int64_t dst_max_sel,
-                                         void *stream) {
-    if (!src_idx || !src_cnt || !src_len || !dst_len || !dst_idx || !dst_cnt || B <= 0 ||
-        H <= 0 || src_max_sel < 1 || src_max_sel > 0x7fffffffLL || dst_max_sel > 0x7fffffffLL)
+namespace {
+
+// Checks shared by the transfer and its stride helper; fills the layout.
+int transfer_layout(const int64_t *src_len, const int64_t *dst_len, int64_t src_max_sel,
+                    sparstar::TransferLayout *ly) {
+    if (!src_len || !dst_len || src_max_sel < 1 || src_max_sel > 0x7fffffffLL)
         return SPARSTAR_EINVAL;
     int64_t Ls = 0, Lt = 0;
     for (int g = 0; g < 4; ++g) {
@@ -287,8 +286,33 @@ SPARSTAR_API int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *
     }
     if (Ls > kMaxTokens || Lt > kMaxTokens) return SPARSTAR_EINVAL;
     if (dst_len[3] > 0 && src_len[3] == 0) return SPARSTAR_EINVAL;
-    if (dst_max_sel < ceil_div(Lt, kBlock) || ceil_div(Ls, kBlock) > sparstar::transfer_max_nkb())
+    if (ceil_div(Ls, kBlock) > sparstar::transfer_max_nkb() ||
+        ceil_div(Lt, kBlock) > sparstar::transfer_max_nkb())
         return SPARSTAR_ESIZE;
+    *ly = sparstar::make_transfer_layout(src_len, dst_len);
+    return SPARSTAR_OK;
+}
+
+}  // namespace
+
+SPARSTAR_API int64_t sparstar_transfer_max_sel(const int64_t *src_len, const int64_t *dst_len,
+                                               int64_t src_max_sel) {
+    sparstar::TransferLayout ly;
+    if (transfer_layout(src_len, dst_len, src_max_sel, &ly) != SPARSTAR_OK) return -1;
+    return sparstar::transfer_max_sel(ly, src_max_sel);
+}
+
+SPARSTAR_API int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt,
+                                         int64_t src_max_sel, int64_t B, int64_t H,
+                                         const int64_t *src_len, const int64_t *dst_len,
+                                         int32_t *dst_idx, int32_t *dst_cnt, int64_t dst_max_sel,
+                                         void *stream) {
+    if (!src_idx || !src_cnt || !dst_idx || !dst_cnt || B <= 0 || H <= 0 ||
+        dst_max_sel > 0x7fffffffLL)
+        return SPARSTAR_EINVAL;
+    sparstar::TransferLayout ly;
+    if (int rc = transfer_layout(src_len, dst_len, src_max_sel, &ly)) return rc;
+    if (dst_max_sel < sparstar::transfer_max_sel(ly, src_max_sel)) return SPARSTAR_ESIZE;
     if (dst_len[3] == 0) return SPARSTAR_OK;
     // list sizes in elements (in double: the product of four checked
     // sizes may not fit in int64)
@@ -297,7 +321,6 @@ SPARSTAR_API int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *
         (double)B * H * ceil_div(dst_len[3], kBlock) * dst_max_sel > 1e12)
         return SPARSTAR_EINVAL;
     if (int rc = device_check()) return rc;
-    const sparstar::TransferLayout ly = sparstar::make_transfer_layout(src_len, dst_len);
     return cuda_status(sparstar::launch_transfer_lists(src_idx, src_cnt, src_max_sel, B * H, ly,
                                                        dst_idx, dst_cnt, dst_max_sel,
                                                        static_cast<cudaStream_t>(stream)));

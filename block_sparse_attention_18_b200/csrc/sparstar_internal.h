@@ -79,5 +79,6 @@ cudaError_t launch_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt
                                   int32_t *dst_idx, int32_t *dst_cnt, int64_t dst_max_sel,
                                   cudaStream_t stream);
 int64_t transfer_max_nkb();
+int64_t transfer_max_sel(const TransferLayout &ly, int64_t src_max_sel);  // host
 
 }  // namespace sparstar

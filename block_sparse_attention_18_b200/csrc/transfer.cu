@@ -14,15 +14,22 @@
 // or when the image of j's centre token lies in a listed source block (the
 // centre of a block of n real tokens starting at a is a + (n - 1) / 2).
 //
-// One warp per target row, eight rows in flight per CTA:
+// The map from a target key block to the source block holding the image of
+// its centre token is the same for every row, so each CTA builds it once in
+// shared memory (-2: forced at the target, -1: no image) and then runs one
+// warp per target row, eight rows in flight, striding over the rows:
 //   1. the source row's list becomes a bitmap in shared memory (one bit per
 //      source key block, entries outside [0, nKB_s) dropped);
-//   2. the 32 lanes test 32 consecutive target blocks at a time: each lane
-//      maps its block's centre token to the source and looks up the bit;
+//   2. the 32 lanes test 32 consecutive target blocks at a time: a map
+//      lookup and a bitmap lookup each;
 //   3. a ballot and a prefix popcount write the kept blocks in ascending
 //      order; the rest of the row is filled with -1.
 // Memory: the source lists are read once and the target lists written once
-// (B*H*nQB_t*max_sel_t int32); the bitmap lookups stay in shared memory.
+// (B*H*nQB_t*max_sel_t int32); the lookups stay in shared memory.
+#include <algorithm>
+#include <functional>
+#include <vector>
+
 #include "sparstar_internal.h"
 
 namespace sparstar {
@@ -30,15 +37,31 @@ namespace {
 
 constexpr int kWarpsPerCta = 8;
 
+// Source block of the image of target block j's centre token; -1 if that
+// token's segment is empty at the source.
+__host__ __device__ inline int32_t centre_image_block(const TransferLayout &ly, int64_t j) {
+    const int64_t a = j * kBlock;
+    const int64_t n_real = ly.Lk_t - a < kBlock ? ly.Lk_t - a : kBlock;
+    const int64_t t = a + (n_real - 1) / 2;  // the block's centre token
+    int g = 0;
+    while (g < 3 && t >= ly.off_t[g] + ly.len_t[g]) ++g;
+    if (ly.len_s[g] == 0) return -1;
+    return (int32_t)((ly.off_s[g] + (t - ly.off_t[g]) * ly.len_s[g] / ly.len_t[g]) / kBlock);
+}
+
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
     transfer_kernel(const int32_t *__restrict__ src_idx, const int32_t *__restrict__ src_cnt,
                     int64_t src_max_sel, TransferLayout ly, int64_t rows,
                     int32_t *__restrict__ dst_idx, int32_t *__restrict__ dst_cnt,
                     int64_t dst_max_sel, int words) {
-    extern __shared__ uint32_t bitmaps[];
+    extern __shared__ uint32_t smem[];
+    int32_t *map = reinterpret_cast<int32_t *>(smem);  // [nKB_t]
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    uint32_t *bm = bitmaps + warp * words;
+    uint32_t *bm = smem + ly.nKB_t + warp * words;
+    for (int j = threadIdx.x; j < ly.nKB_t; j += blockDim.x)
+        map[j] = j < ly.nF_t ? -2 : centre_image_block(ly, j);
+    __syncthreads();
     for (int64_t row = (int64_t)blockIdx.x * kWarpsPerCta + warp; row < rows;
          row += (int64_t)gridDim.x * kWarpsPerCta) {
         const int64_t bh = row / ly.nQB_t;
@@ -66,23 +89,14 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
             const int j = base + lane;
             bool keep = false;
             if (j < ly.nKB_t) {
-                keep = j < ly.nF_t;
-                if (!keep) {
-                    const int64_t a = (int64_t)j * kBlock;
-                    const int64_t n_real = ly.Lk_t - a < kBlock ? ly.Lk_t - a : kBlock;
-                    const int64_t t = a + (n_real - 1) / 2;  // the block's centre token
-                    int g = 0;
-                    while (g < 3 && t >= ly.off_t[g] + ly.len_t[g]) ++g;
-                    if (ly.len_s[g] > 0) {
-                        const int64_t img =
-                            ly.off_s[g] + (t - ly.off_t[g]) * ly.len_s[g] / ly.len_t[g];
-                        const int64_t sb = img / kBlock;
-                        keep = (bm[sb >> 5] >> (sb & 31)) & 1u;
-                    }
-                }
+                const int32_t sb = map[j];
+                keep = sb == -2 || (sb >= 0 && ((bm[sb >> 5] >> (sb & 31)) & 1u));
             }
             const uint32_t ballot = __ballot_sync(0xffffffffu, keep);
-            if (keep) out[n + __popc(ballot & ((1u << lane) - 1u))] = j;
+            const int pos = n + __popc(ballot & ((1u << lane) - 1u));
+            // the host sized the stride for the worst case; the guard only
+            // keeps a wrong stride from writing into the next row
+            if (keep && pos < dst_max_sel) out[pos] = j;
             n += __popc(ballot);
         }
         for (int64_t c = n + lane; c < dst_max_sel; c += 32) out[c] = -1;
@@ -113,7 +127,26 @@ TransferLayout make_transfer_layout(const int64_t *len_s, const int64_t *len_t) 
     return ly;
 }
 
-int64_t transfer_max_nkb() { return 32768; }  // 4 KB of bitmap per warp
+// Source and target key blocks: 4 KB of bitmap per warp and a 128 KB block
+// map, 160 KB of shared memory at most.
+int64_t transfer_max_nkb() { return 32768; }
+
+// Exact worst case of a transferred row's length: every non-forced target
+// block is kept through exactly one source block (the one holding the image
+// of its centre token), so a row that lists m distinct source blocks keeps
+// at most nF_t + the m largest per-source-block counts.
+int64_t transfer_max_sel(const TransferLayout &ly, int64_t src_max_sel) {
+    std::vector<int64_t> hist((size_t)ly.nKB_s, 0);
+    for (int64_t j = ly.nF_t; j < ly.nKB_t; ++j) {
+        const int32_t sb = centre_image_block(ly, j);
+        if (sb >= 0) ++hist[(size_t)sb];
+    }
+    const size_t m = (size_t)std::min<int64_t>(src_max_sel, ly.nKB_s);
+    std::partial_sort(hist.begin(), hist.begin() + m, hist.end(), std::greater<int64_t>());
+    int64_t worst = ly.nF_t < ly.nKB_t ? ly.nF_t : ly.nKB_t;
+    for (size_t c = 0; c < m; ++c) worst += hist[c];
+    return worst;
+}
 
 cudaError_t launch_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt,
                                   int64_t src_max_sel, int64_t BH, const TransferLayout &ly,
@@ -122,16 +155,18 @@ cudaError_t launch_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt
     const int64_t rows = BH * ly.nQB_t;
     if (rows == 0) return cudaSuccess;
     const int words = (int)((ly.nKB_s + 31) / 32);
-    const size_t smem = (size_t)kWarpsPerCta * words * sizeof(uint32_t);
+    const size_t smem = ((size_t)ly.nKB_t + (size_t)kWarpsPerCta * words) * sizeof(uint32_t);
     if (smem > 48 * 1024) {
         const cudaError_t e = cudaFuncSetAttribute(
             transfer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    // Rows are independent and short: enough CTAs for every SM several
-    // times over, each warp striding over the rows.
+    // Each CTA builds the block map, then its warps stride over the rows.
+    // A row is a chain of dependent loads (count, list, bitmap), so up to
+    // eight CTAs per SM keep enough rows in flight; the map (a few integer
+    // divisions per thread) is cheap to rebuild per CTA.
     int64_t ctas = ceil_div(rows, kWarpsPerCta);
-    if (ctas > 148 * 16) ctas = 148 * 16;
+    if (ctas > 148 * 8) ctas = 148 * 8;
     transfer_kernel<<<(unsigned)ctas, kWarpsPerCta * 32, smem, stream>>>(
         src_idx, src_cnt, src_max_sel, ly, rows, dst_idx, dst_cnt, dst_max_sel, words);
     return cudaGetLastError();

@@ -54,6 +54,8 @@ def _load():
     L.sparstar_retained_mass.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, f32, i64, vp, vp,
                                          i64, vp, i64, vp, vp, vp, vp, vp, vp]
     L.sparstar_transfer_lists.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp]
+    L.sparstar_transfer_max_sel.argtypes = [vp, vp, i64]
+    L.sparstar_transfer_max_sel.restype = i64
     L.sparstar_strerror.argtypes = [i32]
     L.sparstar_strerror.restype = ctypes.c_char_p
     L.sparstar_version.restype = i32
@@ -352,21 +354,33 @@ def sparstar_retained_mass(q, k, kv_idx, kv_cnt, n_forced_blocks: int, rows, tau
     return out
 
 
+def _segs(src_len, dst_len):
+    return ((ctypes.c_int64 * 4)(*[int(x) for x in src_len]),
+            (ctypes.c_int64 * 4)(*[int(x) for x in dst_len]))
+
+
+def sparstar_transfer_max_sel(src_len, dst_len, src_max_sel: int) -> int:
+    """Longest row sparstar_transfer_lists can write for these layouts."""
+    ls, lt = _segs(src_len, dst_len)
+    return lib.sparstar_transfer_max_sel(ls, lt, src_max_sel)
+
+
 def sparstar_transfer_lists(kv_idx, kv_cnt, src_len, dst_len, dst_idx=None, dst_cnt=None,
                             stream=None):
     """Diagnostic: block lists of a source scale carried by token position to
     a target scale (mask reuse).  src_len / dst_len: the four segment lengths
-    (text, image_ref, ref, cur) at each scale.  Returns (dst_idx, dst_cnt)
-    with dst_max_sel = the target's key block count unless dst_idx is given."""
+    (text, image_ref, ref, cur) at each scale.  Returns (dst_idx, dst_cnt);
+    dst_idx's row stride is sparstar_transfer_max_sel(...) unless given."""
     _dev(kv_idx, "kv_idx", torch.int32)
     _dev(kv_cnt, "kv_cnt", torch.int32)
     B, H = kv_idx.shape[0], kv_idx.shape[1]
-    ls = (ctypes.c_int64 * 4)(*[int(x) for x in src_len])
-    lt = (ctypes.c_int64 * 4)(*[int(x) for x in dst_len])
-    nKB_t = (sum(int(x) for x in dst_len) + BLOCK - 1) // BLOCK
+    ls, lt = _segs(src_len, dst_len)
     nQB_t = (int(dst_len[3]) + BLOCK - 1) // BLOCK
     if dst_idx is None:
-        dst_idx = torch.empty(B, H, nQB_t, nKB_t, device=kv_idx.device, dtype=torch.int32)
+        stride = lib.sparstar_transfer_max_sel(ls, lt, kv_idx.shape[-1])
+        if stride < 0:
+            raise SparstarError(EINVAL, "sparstar_transfer_lists")
+        dst_idx = torch.empty(B, H, nQB_t, stride, device=kv_idx.device, dtype=torch.int32)
     if dst_cnt is None:
         dst_cnt = torch.empty(B, H, nQB_t, device=kv_idx.device, dtype=torch.int32)
     _dev(dst_idx, "dst_idx", torch.int32)

@@ -344,14 +344,26 @@ int sparstar_retained_mass(const void *q, const void *k, int dtype, int64_t B, i
  *            ascending, unused slots -1
  *   dst_cnt  [B,H,nQB_t] int32 (device, written)
  * The transferred list has no budget of its own (it keeps about the source
- * scale's density); dst_max_sel >= nKB_t (the target's key block count)
- * always suffices and is required.
+ * scale's density); dst_max_sel must be at least
+ * sparstar_transfer_max_sel(src_len, dst_len, src_max_sel), the longest
+ * row any source lists can produce.
  * Errors: SPARSTAR_EINVAL for null pointers, B or H < 1, a negative length,
  * src_len[3] = 0 < dst_len[3], src_max_sel < 1 or more than 2^31 - 1
- * source or target keys; SPARSTAR_ESIZE for dst_max_sel < nKB_t or a source
- * with more than 32768 key blocks.  Nothing is launched on an error, or when
- * dst_len[3] = 0 (no target rows).
+ * source or target keys; SPARSTAR_ESIZE for dst_max_sel below that bound or
+ * a source or target with more than 32768 key blocks.  Nothing is launched on an
+ * error, or when dst_len[3] = 0 (no target rows).  The host computes the
+ * bound on every call (a pass over the target's key blocks).
  */
+/*
+ * Longest transferred row that source lists of stride src_max_sel can give
+ * (host-only; src_len, dst_len as for sparstar_transfer_lists): the
+ * target's forced blocks plus the src_max_sel largest counts of non-forced
+ * target blocks whose centre token has its image in one source block.
+ * Returns -1 for bad arguments (as sparstar_transfer_lists would reject).
+ */
+int64_t sparstar_transfer_max_sel(const int64_t *src_len, const int64_t *dst_len,
+                                  int64_t src_max_sel);
+
 int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt, int64_t src_max_sel,
                             int64_t B, int64_t H, const int64_t *src_len, const int64_t *dst_len,
                             int32_t *dst_idx, int32_t *dst_cnt, int64_t dst_max_sel,

@@ -581,7 +581,8 @@ static int64_t orc_image(int64_t t, const int64_t *off_s, const int64_t *off_t,
  * Output kv_idx_t [B,H,nQB_t,max_sel_t]: the kept blocks ascending, unused
  * slots -1; kv_cnt_t [B,H,nQB_t].  Source entries outside [0, nKB_s) are
  * ignored; a source count above max_sel_s is read as max_sel_s.
- * Returns 0; -1 if max_sel_t < nKB_t; -2 if len_s[3] = 0 < len_t[3]. */
+ * Returns 0; -1 if a row keeps more than max_sel_t blocks (nothing past
+ * the stride is written); -2 if len_s[3] = 0 < len_t[3]. */
 int orc_transfer_lists(const int32_t *idx_s, const int32_t *cnt_s, int64_t max_sel_s,
                        int64_t B, int64_t H, const int64_t *len_s, const int64_t *len_t,
                        int32_t *idx_t, int32_t *cnt_t, int64_t max_sel_t)
@@ -596,9 +597,9 @@ int orc_transfer_lists(const int32_t *idx_s, const int32_t *cnt_s, int64_t max_s
     const int64_t nKB_s = orc_nblocks(Lk_s), nKB_t = orc_nblocks(Lk_t);
     const int64_t nQB_s = orc_nblocks(len_s[3]), nQB_t = orc_nblocks(len_t[3]);
     const int64_t nF_t = orc_forced_blocks(len_t[0], len_t[1]);
-    if (max_sel_t < nKB_t) return -1;
     if (len_t[3] > 0 && len_s[3] == 0) return -2;
-#pragma omp parallel for schedule(dynamic, 4)
+    int overflow = 0;
+#pragma omp parallel for schedule(dynamic, 4) reduction(| : overflow)
     for (int64_t row = 0; row < B * H * nQB_t; ++row) {
         const int64_t bh = row / nQB_t;
         const int64_t i = row % nQB_t;
@@ -627,11 +628,15 @@ int orc_transfer_lists(const int32_t *idx_s, const int32_t *cnt_s, int64_t max_s
                         }
                 }
             }
-            if (keep) idx_t[row * max_sel_t + n++] = (int32_t)j;
+            if (keep) {
+                if (n < max_sel_t) idx_t[row * max_sel_t + n] = (int32_t)j;
+                ++n;
+            }
         }
+        if (n > max_sel_t) overflow = 1;
         for (int64_t c = n; c < max_sel_t; ++c)
             idx_t[row * max_sel_t + c] = -1;
         cnt_t[row] = (int32_t)n;
     }
-    return 0;
+    return overflow ? -1 : 0;
 }

@@ -194,7 +194,14 @@ def test_transfer_lists_argument_errors(sp):
     assert call(src=NUL) == sp.EINVAL
     assert call(src=seg(128, 0, -1, 256)) == sp.EINVAL
     assert call(src=seg(128, 0, 256, 0)) == sp.EINVAL  # target queries without a source
-    assert call(dst_max_sel=8) == sp.ESIZE  # below nKB_t
+    # Hand-derived stride bound: nF_t = 1; the 8 other target blocks have
+    # their centre images two by two in source blocks 1, 2, 3, 4.
+    assert sp.sparstar_transfer_max_sel([128, 0, 256, 256], [128, 0, 512, 512], 4) == 9
+    assert sp.sparstar_transfer_max_sel([128, 0, 256, 256], [128, 0, 512, 512], 2) == 5
+    assert sp.sparstar_transfer_max_sel([128, 0, 256, 256], [128, 0, 512, 512], 1) == 3
+    assert sp.sparstar_transfer_max_sel([128, 0, 256, 0], [128, 0, 512, 512], 1) == -1
+    assert call(dst_max_sel=8) == sp.ESIZE  # below the bound (9)
     assert call(src=seg(128, 0, 32768 * 128, 256)) == sp.ESIZE  # source bitmap limit
+    assert call(dst=seg(128, 0, 32768 * 128, 512)) == sp.ESIZE  # target block-map limit
     # no target rows: nothing to do, nothing launched, even without a device
-    assert call(dst=seg(128, 0, 512, 0), dst_max_sel=5) == sp.OK
+    assert call(dst=seg(128, 0, 512, 0), dst_max_sel=9) == sp.OK

@@ -54,10 +54,12 @@ def _random_lists(rng, B, H, nQB, nKB, max_sel, count=None, p_invalid=0.0):
 
 
 def _both(sp, orc, idx, cnt, len_s, len_t):
-    want_idx, want_cnt = orc.transfer_lists(idx, cnt, len_s, len_t)
     got_idx, got_cnt = sp.sparstar_transfer_lists(torch.from_numpy(idx).cuda(),
                                                   torch.from_numpy(cnt).cuda(), len_s, len_t)
     torch.cuda.synchronize()
+    stride = sp.sparstar_transfer_max_sel(len_s, len_t, idx.shape[-1])
+    assert got_idx.shape[-1] == stride
+    want_idx, want_cnt = orc.transfer_lists(idx, cnt, len_s, len_t, max_sel_t=stride)
     assert np.array_equal(got_cnt.cpu().numpy(), want_cnt)
     assert np.array_equal(got_idx.cpu().numpy(), want_idx)
     return want_idx, want_cnt
@@ -149,3 +151,34 @@ def test_attention_over_transferred_lists(sp, orc):
     nF = _nb(tgt.text)
     sel_t = nF + int(np.ceil(tgt.density * (tgt.nKB - nF)))
     assert tcnt.mean() > sel_t
+
+
+@pytest.mark.parametrize("pair", PAIRS[:3], ids=lambda p: "%s->%s" % p)
+def test_worst_case_rows_reach_the_stride_bound(sp, orc, pair):
+    # The bound is the forced prefix plus the largest per-source-block
+    # counts.  The counts come from the oracle with single-block lists; a
+    # row that lists the m blocks with the largest counts must reach it.
+    ws, wt = synth.WORKLOADS[pair[0]], synth.WORKLOADS[pair[1]]
+    seg_s, seg_t = _seg(ws), _seg(wt)
+    nF_t = _nb(wt.text + wt.image_ref)
+    one = np.tile(np.arange(ws.nKB, dtype=np.int32).reshape(1, ws.nKB, 1, 1), (1, 1, ws.nQB, 1))
+    _, c1 = orc.transfer_lists(one, np.ones((1, ws.nKB, ws.nQB), np.int32), seg_s, seg_t)
+    per_block = c1[0, :, 0] - nF_t  # target blocks kept through each source block
+    m = 40
+    top = np.sort(np.argsort(-per_block, kind="stable")[:m]).astype(np.int32)
+    assert sp.sparstar_transfer_max_sel(seg_s, seg_t, m) == nF_t + int(np.sort(per_block)[-m:].sum())
+    idx = np.tile(top, (1, 1, ws.nQB, 1))
+    cnt = np.full((1, 1, ws.nQB), m, np.int32)
+    got_idx, got_cnt = _both(sp, orc, idx, cnt, seg_s, seg_t)
+    assert (got_cnt == got_idx.shape[-1]).all()
+
+
+def test_target_at_the_block_map_limit(sp, orc):
+    # 32768 target key blocks, the largest block map a CTA holds
+    len_s = [128, 0, 50000, 700]
+    len_t = [128, 0, 32768 * 128 - 128 - 900, 900]
+    assert _nb(sum(len_t)) == 32768
+    nKB_s = _nb(sum(len_s))
+    rng = np.random.default_rng(77)
+    idx, cnt = _random_lists(rng, 1, 2, _nb(len_s[3]), nKB_s, 60)
+    _both(sp, orc, idx, cnt, len_s, len_t)

@@ -190,10 +190,13 @@ def test_invariants_and_empty_source_lists(orc):
 
 
 def test_error_returns(orc):
-    idx = np.zeros((1, 1, 1, 2), np.int32)
-    cnt = np.ones((1, 1, 1), np.int32)
-    with pytest.raises(ValueError):  # max_sel_t below nKB_t
+    # source cur block 1 maps onto target blocks 1..4: a row of 5 > stride 2
+    idx = np.array([[[[1, 0]]]], np.int32)
+    cnt = np.full((1, 1, 1), 2, np.int32)
+    with pytest.raises(ValueError):
         orc.transfer_lists(idx, cnt, [128, 0, 0, 100], [128, 0, 0, 400], max_sel_t=2)
+    idx_t, cnt_t = orc.transfer_lists(idx, cnt, [128, 0, 0, 100], [128, 0, 0, 400], max_sel_t=5)
+    assert list(idx_t[0, 0, 0]) == [0, 1, 2, 3, 4] and cnt_t[0, 0, 0] == 5
     with pytest.raises(ValueError):  # no query tokens at the source
         orc.transfer_lists(np.zeros((1, 1, 0, 2), np.int32), np.zeros((1, 1, 0), np.int32),
                            [128, 0, 0, 0], [128, 0, 0, 400])
