@@ -65,7 +65,7 @@ constexpr int kOffStage = 3 * kTileBytes;
 constexpr int kOffBar = kOffStage + kStages * kTileBytes;
 struct Bars {
     uint64_t q_full;
-    uint64_t st_full[kStages];
+    uint64_t st_full[kStages][2];  // [stage][use & 1]
     uint64_t st_empty[kStages];
     uint64_t s_full[2];   // per query block
     uint64_t s_free[2];
@@ -340,6 +340,19 @@ __device__ __forceinline__ int slot_k(int x, int j, int nA, int nB) {
 __device__ __forceinline__ int slot_v(int x, int j, int nA, int nB) {
     return steps_before(j + 2, nA, nB) + steps_before(j, nA, nB) + ((x == 1 && j < nA) ? 1 : 0);
 }
+// The QK warp consumes the key tiles and the PV warp the value tiles, so a
+// stage's previous occupant (slot e - kStages) can be the other warp's tile
+// and still be in flight when this warp tests slot e; with one full barrier
+// per stage a parity test cannot tell that state from "slot e landed".
+// Each stage therefore has two full barriers, for its even and its odd
+// uses: slot e waits on barrier (e / kStages) & 1 for that barrier's phase
+// e / (2 kStages), whose previous phase is slot e - 2 kStages.  That slot
+// has always landed before the test (the waits between the roles guarantee
+// it for every pair of list lengths; tests/test_ring_protocol.py checks
+// the happens-before chains), so the wait is exact.
+__device__ __forceinline__ uint32_t ring_parity(int e) {
+    return (uint32_t)(e / (2 * kStages)) & 1u;
+}
 // ------------------------------------------------------------------ kernel
 
 __global__ void __maxnreg__(168)
@@ -370,7 +383,11 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     cntB = cntB < 0 ? 0 : (cntB > max_sel ? max_sel : cntB);
 
     const uint32_t bar_q = smem_addr(&bars->q_full);
-    auto bar_full = [&](int s) { return smem_addr(&bars->st_full[s]); };
+    // Ring slot e is use e / kStages of stage e % kStages; each stage has two
+    // full barriers that alternate between its uses (see ring_wait).
+    auto bar_full = [&](int e) {
+        return smem_addr(&bars->st_full[e % kStages][(e / kStages) & 1]);
+    };
     auto bar_empty = [&](int s) { return smem_addr(&bars->st_empty[s]); };
     auto bar_s = [&](int x) { return smem_addr(&bars->s_full[x]); };
     auto bar_sfree = [&](int x) { return smem_addr(&bars->s_free[x]); };
@@ -385,7 +402,8 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (lane == 0) {
             mbar_init(bar_q, 1);
             for (int s = 0; s < kStages; ++s) {
-                mbar_init(bar_full(s), 1);
+                mbar_init(smem_addr(&bars->st_full[s][0]), 1);
+                mbar_init(smem_addr(&bars->st_full[s][1]), 1);
                 mbar_init(bar_empty(s), 1);
             }
             for (int x = 0; x < 2; ++x) {
@@ -467,9 +485,9 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const int kb = next_valid(lx, cx, cr, nKB);
                     const uint32_t dst = base + kOffStage + stage * kTileBytes;
                     const CUtensorMap *map = is_v ? &tmV : &tmK;
-                    mbar_expect_tx(bar_full(stage), kTileBytes);
-                    tma_load_3d(dst, map, bar_full(stage), 0, kb * kBlock, bh, pol_kv);
-                    tma_load_3d(dst + kPanelBytes, map, bar_full(stage), 64, kb * kBlock, bh,
+                    mbar_expect_tx(bar_full(e), kTileBytes);
+                    tma_load_3d(dst, map, bar_full(e), 0, kb * kBlock, bh, pol_kv);
+                    tma_load_3d(dst + kPanelBytes, map, bar_full(e), 64, kb * kBlock, bh,
                                 pol_kv);
                     ++e;
                 }
@@ -479,7 +497,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             drain_wait(bar_q, 0);
             const int first = e > kStages ? e - kStages : 0;
             for (int i = first; i < e; ++i)
-                drain_wait(bar_full(i % kStages), (uint32_t)(i / kStages) & 1u);
+                drain_wait(bar_full(i), ring_parity(i));
         }
     } else if (warp == kMmaWarp) {
         // -------------------------------------------- S = Q K^T MMA issuer
@@ -494,8 +512,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (!ok || j >= (x == 0 ? nA : nB)) continue;
                 const int e = slot_k(x, j, nA, nB);
                 const int stage = e % kStages;
-                if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag,
-                               status)) {
+                if (!wait_warp(bar_full(e), ring_parity(e), abort_flag, status)) {
                     ok = false;
                     break;
                 }
@@ -542,8 +559,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tc_fence_after();  // orders an O rescale (tcgen05.st) before the MMA
                 const int e = slot_v(x, j, nA, nB);
                 const int stage = e % kStages;
-                if (!wait_warp(bar_full(stage), (uint32_t)(e / kStages) & 1u, abort_flag,
-                               status)) {
+                if (!wait_warp(bar_full(e), ring_parity(e), abort_flag, status)) {
                     ok = false;
                     break;
                 }
