@@ -638,12 +638,16 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 for (int c = 0; c < kBlock; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
+            // four chains: s[0..3], then two quads per step (s[4..123]),
+            // then the last quad
             float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int c = 4; c < kBlock; c += 8) {
+            for (int c = 4; c + 8 <= kBlock; c += 8) {
 #pragma unroll
                 for (int t = 0; t < 4; ++t) mx[t] = max3f(mx[t], s[c + t], s[c + 4 + t]);
             }
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mx[t] = fmaxf(mx[t], s[kBlock - 4 + t]);
             const float m_tile = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
             const float m_new = fmaxf(m_ref, m_tile);
             bool p_free = false;  // the P buffer is free for this hand-off
