@@ -609,8 +609,13 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         float m_ref = -INFINITY, l = 0.0f;
         bool ok = true;
         int cur = 0;
+        const bool has_tail = (Lk % kBlock) != 0;
         for (int j = 0; j < nx; ++j) {
-            const int kb = next_valid(x ? listB : listA, x ? cntB : cntA, cur, nKB);
+            // Only a partial last key block needs masking, so the list is
+            // read only when Lk is not a multiple of the block size (else its
+            // global load would sit on the path to the tile max).
+            const int kb =
+                has_tail ? next_valid(x ? listB : listA, x ? cntB : cntA, cur, nKB) : 0;
             if (!wait_warp(bar_s(x), (uint32_t)j & 1u, abort_flag, status)) {
                 ok = false;
                 break;
@@ -633,7 +638,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             tc_fence_before();
             mbar_arrive(bar_sfree(x));
             const int valid = Lk - kb * kBlock;  // keys of this tile that exist
-            if (valid < kBlock) {
+            if (has_tail && valid < kBlock) {
 #pragma unroll
                 for (int c = 0; c < kBlock; ++c)
                     if (c >= valid) s[c] = -INFINITY;
