@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # SHA-256 of the kernel source it was taken on; reported only while the
 # source is unchanged.
 ATTN_TRAFFIC = {
-    "source_sha256": "0632efc1c668b3d27f5c136fa75c08b52f198bb3b36dd448df1832fbb168e0ba",
-    "bytes_per_launch": 3525226240 + 294929408,  # largest workload, one launch
+    "source_sha256": "0b3a76d19a5277b353332cf2912b53afd025063a0efb2cdc1b49ad16c821344f",
+    "bytes_per_launch": 3583543808 + 298071040,  # largest workload, one launch
 }
 
 
