@@ -3,7 +3,8 @@
 // pith.science review, "Extended reading notes / Core claim": reusing a
 // block-selection pattern across scales loses retained attention mass, which
 // is why the method recomputes the selection at every scale; Figure 1 of the
-// review: a reused support misses blocks that become active).
+// review: blocks that matter at the new scale can lie outside a mask carried
+// over from the earlier one).
 //
 // The pages give no map between two scales' token positions.  Reading: the
 // block mask is resampled by nearest neighbour along each key segment g of

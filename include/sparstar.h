@@ -319,8 +319,8 @@ int sparstar_retained_mass(const void *q, const void *k, int dtype, int64_t B, i
  * scales that the method argues against.  Source: pith.science review of
  * SparSTAR, "Extended reading notes / Core claim" (reusing a block-selection
  * pattern across scales loses retained attention mass, so the selection is
- * recomputed at every scale) and Figure 1 (a reused support misses blocks
- * that become active).  The pages give no map between two scales' token
+ * recomputed at every scale) and Figure 1 (a carried-over mask can leave
+ * out blocks that matter at the new scale).  The pages give no map between two scales' token
  * positions; this call resamples the block mask by nearest neighbour
  * along the token order, the plainest reading:
  *   - keys at both scales are the segments [text | image_ref | ref | cur];

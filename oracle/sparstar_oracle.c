@@ -561,10 +561,10 @@ static int64_t orc_image(int64_t t, const int64_t *off_s, const int64_t *off_t,
  * the "reuse" that the method argues against ([R-core]: reusing a
  * block-selection pattern across scales loses retained attention mass, so
  * the selection is recomputed at every scale; the review's Figure 1: a
- * reused support misses blocks that become active at the new scale).  The
- * pages give no map between two scales' token positions; the reading used
- * (listed in the design notes) resamples the block mask by nearest
- * neighbour along the token order:
+ * mask carried over from an earlier scale can leave out blocks that matter
+ * at the new one).  The pages give no map between two scales' token
+ * positions; the reading used (listed in the design notes) resamples the
+ * block mask by nearest neighbour along the token order:
  *   - keys at both scales are the segments [text | image_ref | ref | cur];
  *     segment g has len_s[g] tokens at the source and len_t[g] at the
  *     target (queries are the cur segment);

@@ -3,7 +3,8 @@
 Sources: pith.science review of SparSTAR, "Extended reading notes / Core
 claim" (reusing a block-selection pattern across scales loses retained
 attention mass; the method recomputes the selection at every scale) and
-Figure 1 (a reused support misses blocks that become active).  The pages give
+Figure 1 (a carried-over mask can leave out blocks that matter at the new
+scale).  The pages give
 no map between the token positions of two scales.  The reading pinned here
 resamples the block mask by nearest neighbour along each key segment (text,
 image_ref, ref, cur):
