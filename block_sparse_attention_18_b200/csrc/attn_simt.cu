@@ -1,7 +1,7 @@
 // Step 3 for fp32 inputs (D 64 or 128) and bf16 with D = 64: forward
 // attention over the listed 128 x 128 tiles in fp32 FFMA (SparSTAR,
-// pith.science review, "What carries the argument": the chosen blocks are
-// executed through a forward-only attention path).
+// pith.science review, "What carries the argument": only the chosen blocks
+// are attended, and only forward).
 //
 // fp32 inputs must meet a 1e-4 max-abs tolerance, which rules out TF32
 // tensor cores; this kernel keeps every product and sum in fp32.  It is the

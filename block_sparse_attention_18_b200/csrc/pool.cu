@@ -1,6 +1,6 @@
 // Step 1 — 128-token block mean pooling of Q or K (SparSTAR, pith.science
-// review, "What carries the argument": block-averaged query and key vectors
-// over contiguous 128-token blocks).
+// review, "What carries the argument": the score uses the mean query and the
+// mean key of each run of 128 consecutive tokens).
 //
 // One CTA per (b, h, block).  The block's rows are 128 x D elements; each
 // row is split into 16-byte chunks.  Thread (stripe r, chunk c) sums, in

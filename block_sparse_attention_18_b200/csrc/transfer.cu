@@ -1,8 +1,8 @@
 // Diagnostic — block lists reused across scales: the lists selected at a
 // source scale, carried by token position to a target scale (SparSTAR,
-// pith.science review, "Extended reading notes / Core claim": reusing a
-// block-selection pattern across scales loses retained attention mass, which
-// is why the method recomputes the selection at every scale; Figure 1 of the
+// pith.science review, "Extended reading notes / Core claim": a selection
+// carried from one scale to another keeps less of the attention mass than a
+// fresh one, which is why the method selects anew at every scale; Figure 1 of the
 // review: blocks that matter at the new scale can lie outside a mask carried
 // over from the earlier one).
 //

@@ -8,8 +8,8 @@
  *   1. average Q and K over contiguous 128-token blocks;
  *   2. score every (query block i, key block j) pair as
  *      S_ij = tau * qbar_i^T kbar_j, tau = D^-1/2 (the paper's Eq. 2), keep
- *      the text blocks (and, for Clip 1, the image-pyramid reference blocks)
- *      by force, and keep the top ceil(density * C) of the remaining C
+ *      every block holding text (and, in Clip 1, the last image-pyramid
+ *      reference) whatever its score, and keep the top ceil(density * C) of the remaining C
  *      reference and current-scale blocks, ranked jointly;
  *   3. run a forward-only attention over the selected 128 x 128 tiles only,
  *      described by a forward block list (per-row count + key-block index
@@ -20,13 +20,13 @@
  *              "What carries the argument": block-averaged q and k over
  *              contiguous 128-token blocks, the score S_ij = tau qbar_i^T
  *              kbar_j (Eq. 2), the block-average identity, text / Clip-1
- *              reference retained dense, joint ranking of reference and
+ *              reference always kept, one ranking shared by reference and
  *              current blocks under the density schedule, forward-only
  *              mask fields (FastFlex).
- *   abstract   SparSTAR abstract (mlsanity.com/paper/2608.10519): per scale
- *              and head, contiguous key blocks are scored from the current
- *              query and key activations and the selected blocks run through
- *              a forward-only sparse path.
+ *   abstract   SparSTAR abstract (mlsanity.com/paper/2608.10519): the
+ *              block scores are computed anew at each scale and head from
+ *              that scale's own Q and K, and only the chosen blocks go
+ *              through the (forward-only) sparse attention.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -113,9 +113,9 @@ int sparstar_block_score(const float *qbar, const float *kbar, int64_t B, int64_
 /*
  * sparstar_forced_blocks — host only.  Number of leading key blocks that
  * hold at least one text or Clip-1 image-reference token:
- * ceil((text_len + image_ref_len) / 128).  Source: [R-carry] — text, and for
- * Clip 1 the final image-pyramid reference, are never dropped from the
- * attention.  Returns -1 for negative lengths.
+ * ceil((text_len + image_ref_len) / 128).  Source: [R-carry] — the text
+ * tokens, and in Clip 1 the last image-pyramid reference, always take part
+ * in the attention.  Returns -1 for negative lengths.
  */
 int64_t sparstar_forced_blocks(int64_t text_len, int64_t image_ref_len);
 
@@ -317,9 +317,9 @@ int sparstar_retained_mass(const void *q, const void *k, int dtype, int64_t B, i
  * sparstar_transfer_lists — diagnostic: the block lists of a source scale
  * carried by token position to a target scale, i.e. the mask reuse across
  * scales that the method argues against.  Source: pith.science review of
- * SparSTAR, "Extended reading notes / Core claim" (reusing a block-selection
- * pattern across scales loses retained attention mass, so the selection is
- * recomputed at every scale) and Figure 1 (a carried-over mask can leave
+ * SparSTAR, "Extended reading notes / Core claim" (a selection carried from
+ * one scale to another keeps less attention mass than a fresh one, so the
+ * method selects anew at every scale) and Figure 1 (a carried-over mask can leave
  * out blocks that matter at the new scale).  The pages give no map between two scales' token
  * positions; this call resamples the block mask by nearest neighbour
  * along the token order, the plainest reading:

@@ -13,8 +13,8 @@
  *              contiguous 128-token blocks taken in the order the attention
  *              kernel walks them, block-averaged q and k,
  *              S_ij = tau * qbar_i^T kbar_j with
- *              tau = D^-1/2, the block-average identity, text (and, for
- *              Clip 1, the final image-pyramid reference) retained dense,
+ *              tau = D^-1/2, the block-average identity, the text (and, in
+ *              Clip 1, the last image-pyramid reference) always kept,
  *              reference and current blocks ranked jointly under a density
  *              schedule, forward-only block mask (per-row count + index
  *              list, no reverse index).
@@ -26,10 +26,10 @@
  *   [R-settle] same review, "What would settle it": replacing the block
  *              score by the exact token-wise Top-K at the same densities is
  *              the test of whether block aggregation costs fidelity.
- *   [R-abs]    SparSTAR abstract (mlsanity.com/paper/2608.10519): scores
- *              contiguous key blocks per scale and head from the current
- *              query and key activations; executes selected blocks through
- *              a forward-only sparse path.
+ *   [R-abs]    SparSTAR abstract (mlsanity.com/paper/2608.10519): block
+ *              scores computed anew per scale and head from that scale's
+ *              own Q and K; only the chosen blocks are attended, forward
+ *              only.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   - One block grid over the concatenated keys, one over the queries;
@@ -251,8 +251,8 @@ static int orc_int_cmp(const void *pa, const void *pb)
 }
 
 /* One row of the clip-aware block Top-K ([R-carry] policy, [R-ref]):
- * forced blocks 0..nF-1 are kept; the candidates nF..nKB-1 (preceding-clip
- * reference and current-scale blocks together) are sorted by score and the
+ * forced blocks 0..nF-1 are kept; the candidates nF..nKB-1 (blocks of the
+ * earlier clip's context and of this scale, in one pool) are sorted by score and the
  * first k kept; the list is written forced-first, then the chosen
  * candidates in ascending block order. */
 static void orc_select_row(const double *scores, int64_t nKB, int64_t nF,
@@ -558,9 +558,9 @@ static int64_t orc_image(int64_t t, const int64_t *off_s, const int64_t *off_t,
 }
 
 /* The block lists of a source scale carried to a target scale by position:
- * the "reuse" that the method argues against ([R-core]: reusing a
- * block-selection pattern across scales loses retained attention mass, so
- * the selection is recomputed at every scale; the review's Figure 1: a
+ * the "reuse" that the method argues against ([R-core]: a selection
+ * carried from one scale to another keeps less of the attention mass than
+ * a fresh one, so the method selects anew at every scale; the review's Figure 1: a
  * mask carried over from an earlier scale can leave out blocks that matter
  * at the new one).  The pages give no map between two scales' token
  * positions; the reading used (listed in the design notes) resamples the

@@ -2,8 +2,8 @@
 reuse) with the oracle, bit for bit, and of attention over transferred lists.
 
 Source: pith.science review of SparSTAR, "Extended reading notes / Core
-claim" (reusing a block-selection pattern across scales loses retained
-attention mass) and Figure 1 (a carried-over mask can leave out blocks that
+claim" (a selection carried from one scale to another keeps less attention
+mass than a fresh one) and Figure 1 (a carried-over mask can leave out blocks that
 matter at the new scale).
 The map between scales is the proportional per-segment reading that the
 oracle's pins fix.

@@ -1,8 +1,8 @@
 """Pins of the oracle's cross-scale list transfer (mask reuse; CPU only).
 
 Sources: pith.science review of SparSTAR, "Extended reading notes / Core
-claim" (reusing a block-selection pattern across scales loses retained
-attention mass; the method recomputes the selection at every scale) and
+claim" (a selection carried from one scale to another keeps less attention
+mass than a fresh one; the method selects anew at every scale) and
 Figure 1 (a carried-over mask can leave out blocks that matter at the new
 scale).  The pages give
 no map between the token positions of two scales.  The reading pinned here
