@@ -131,3 +131,28 @@ def test_uneven_list_lengths_within_pairs(sp, orc, seed):
             idx[0, h, i, :len(lst)] = lst
             cnt[0, h, i] = len(lst)
     _run(sp, orc, w, idx=idx, cnt=cnt, expect_status=sp.STATUS_BAD_INDEX if bad else 0)
+
+
+def test_every_list_length_pair_up_to_12(sp, orc):
+    """Every pair of list lengths (nA, nB) with 0 <= nA, nB <= 12 in one
+    launch: 19 heads x 9 query-block pairs, the pair (A, B) of head h, pair p
+    taking combination 9h + p.  These are the pairs the ring's happens-before
+    model covers (tests/test_ring_protocol.py); on the GPU each runs the
+    producer order, the slot closed forms and the alternating full barriers
+    through its own mix of key and value tiles."""
+    w = synth.custom(H=19, D=128, dtype="bf16", text=128, ref=640, cur=18 * 128,
+                     density=1.0, seed=77)
+    nQB, nKB = w.nQB, w.nKB
+    assert nQB == 18 and nKB >= 12
+    rng = np.random.default_rng(12)
+    combos = [(a, b) for a in range(13) for b in range(13)]
+    idx = np.full((1, w.H, nQB, 12), -1, np.int32)
+    cnt = np.zeros((1, w.H, nQB), np.int32)
+    for c, (na, nb) in enumerate(combos):
+        h, p = divmod(c, 9)
+        for i, n in ((2 * p, na), (2 * p + 1, nb)):
+            lst = np.sort(rng.choice(nKB, size=n, replace=False))
+            idx[0, h, i, :n] = lst
+            cnt[0, h, i] = n
+    rows = parity.sample_rows(w.B, w.H, w.Lq, per_head_blocks=18, rows_per_block=4, seed=5)
+    _run(sp, orc, w, idx=idx, cnt=cnt, rows=rows)
