@@ -78,7 +78,11 @@ def attention_flops(kv_idx: np.ndarray, kv_cnt: np.ndarray, Lq: int, Lk: int, D:
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while running."""
+    """Samples nvidia-smi clocks and throttle reasons every 50 ms while
+    running.  Each sample keeps its host arrival time, so that summary()
+    can keep only the samples taken inside a given window (the timed
+    region); started ahead of the region, it is already sampling when the
+    region begins."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -87,7 +91,8 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
-        self.lines = []
+        self.lines = []  # (host arrival time, csv line)
+        self.window = None
 
     def _gpu_id(self):
         try:
@@ -100,7 +105,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self._gpu_id(), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -110,7 +115,13 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def wait_first(self, timeout_s=3.0):
+        """Block (bounded) until the sampler has produced a line."""
+        t_end = time.monotonic() + timeout_s
+        while self.proc is not None and not self.lines and time.monotonic() < t_end:
+            time.sleep(0.01)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -124,7 +135,9 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for t, line in self.lines:
+            if self.window is not None and not (self.window[0] <= t <= self.window[1]):
+                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) != 7:
                 continue
@@ -380,9 +393,11 @@ def run_gpu(args, world, rank, local):
             stream.wait_stream(cap)
             graph.replay()  # upload; not timed
             torch.cuda.synchronize(device)
-        barrier(world, device)
-        torch.cuda.synchronize(device)
         with ClockSampler(local) as clk_:
+            clk_.wait_first()
+            barrier(world, device)
+            torch.cuda.synchronize(device)
+            h0 = time.monotonic()
             t0.record(stream)
             if graph is not None:
                 graph.replay()
@@ -391,6 +406,11 @@ def run_gpu(args, world, rank, local):
                     step_fn(stream, evs[s_i])
             t1.record(stream)
             torch.cuda.synchronize(device)
+            h1 = time.monotonic()
+            time.sleep(0.06)  # the sample taken at the region's end arrives
+            # samples that arrive within one interval after the region ends
+            # were taken inside it
+            clk_.window = (h0, h1 + 0.05)
         barrier(world, device)
         total = max_over_ranks(t0.elapsed_time(t1), world, device)
         per_ = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(n_names)]
