@@ -504,6 +504,9 @@ def run_gpu(args, world, rank, local):
         "config": workload_config(w, world),
         "attn_ms": per["attn"], "attn_tflops": attn_tflops,
         "attn_pct_of_bf16_peak": {"measured_burst": 100 * attn_tflops / peaks["bf16_tflops"],
+                                  "measured_sustained": (
+                                      100 * attn_tflops / peaks["bf16_tflops_sustained"]
+                                      if peaks.get("bf16_tflops_sustained") else None),
                                   "datasheet_2250": 100 * attn_tflops / DATASHEET_BF16_TFLOPS},
         "chain": args.chain, "graph": bool(fused and args.graph),
         "kernel_ms": per, "selection_share_pct": 100 * sel_ms / sum(per.values()),
