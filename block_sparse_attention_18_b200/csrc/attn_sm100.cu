@@ -362,7 +362,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                        int nPair, float tau, const int32_t *__restrict__ kv_idx,
                        const int32_t *__restrict__ kv_cnt, int max_sel,
                        __nv_bfloat16 *__restrict__ out, float *__restrict__ lse,
-                       int32_t *__restrict__ status) {
+                       int32_t *__restrict__ status, int withhold_kv) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -468,7 +468,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             bool ok = true;
             // Groups K(0), K(1), V(0), K(2), V(1), K(3), ...: group g > 0
             // is K((g+1)/2) when odd, V(g/2-1) when even.
-            for (int g = 0; g <= 2 * nmax && ok; ++g) {
+            // withhold_kv (a test hook): no key or value tile is loaded, so
+            // the first wait on the ring runs out and every role takes its
+            // abort path.
+            for (int g = 0; g <= 2 * nmax && ok && !withhold_kv; ++g) {
                 const bool is_v = g > 0 && (g & 1) == 0;
                 const int j = g == 0 ? 0 : (is_v ? g / 2 - 1 : (g + 1) / 2);
                 for (int x = 0; x < 2 && ok; ++x) {
@@ -844,7 +847,7 @@ bool encode(CUtensorMap *map, const void *ptr, int64_t BH, int64_t L) {
 int launch_attn_sm100(const void *q, const void *k, const void *v, int64_t BH, int64_t Lq,
                            int64_t Lk, float tau, const int32_t *kv_idx, const int32_t *kv_cnt,
                            int64_t max_sel, void *out, float *lse, int32_t *status,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool withhold_kv) {
     CUtensorMap mq, mk, mv;
     if (!encode(&mq, q, BH, Lq) || !encode(&mk, k, BH, Lk) || !encode(&mv, v, BH, Lk))
         return SPARSTAR_ECUDA;
@@ -855,7 +858,7 @@ int launch_attn_sm100(const void *q, const void *k, const void *v, int64_t BH, i
     const int64_t nPair = ceil_div(nQB, 2);
     attn_sm100_kernel<<<(unsigned)(BH * nPair), kThreads, kSmemBytes, stream>>>(
         mq, mk, mv, (int)Lq, (int)Lk, (int)nQB, (int)nKB, (int)nPair, tau, kv_idx, kv_cnt,
-        (int)max_sel, static_cast<__nv_bfloat16 *>(out), lse, status);
+        (int)max_sel, static_cast<__nv_bfloat16 *>(out), lse, status, withhold_kv ? 1 : 0);
     return cudaGetLastError() == cudaSuccess ? SPARSTAR_OK : SPARSTAR_ECUDA;
 }
 

@@ -325,3 +325,22 @@ SPARSTAR_API int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *
                                                        dst_idx, dst_cnt, dst_max_sel,
                                                        static_cast<cudaStream_t>(stream)));
 }
+
+SPARSTAR_API int sparstar_test_attn_timeout(const void *q, const void *k, const void *v,
+                                            int64_t B, int64_t H, int64_t Lq, int64_t Lk,
+                                            const int32_t *kv_idx, const int32_t *kv_cnt,
+                                            int64_t max_sel, void *out, int32_t *status,
+                                            void *stream) {
+    if (!q || !k || !v || !out || !kv_cnt || !status || B <= 0 || H <= 0 || Lq <= 0 ||
+        Lk <= 0 || max_sel < 0 || (max_sel > 0 && !kv_idx))
+        return SPARSTAR_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return SPARSTAR_EINVAL;
+    if (Lq > kMaxTokens || Lk > kMaxTokens || max_sel > 0x7fffffffLL ||
+        B * H * ceil_div(Lq, kBlock) > kMaxGrid || B * H > 0x7fffffffLL)
+        return SPARSTAR_EINVAL;
+    if (int rc = device_check()) return rc;
+    return sparstar::launch_attn_sm100(q, k, v, B * H, Lq, Lk, 0.0883883476f, kv_idx, kv_cnt,
+                                       max_sel, out, nullptr, status,
+                                       static_cast<cudaStream_t>(stream), true);
+}

@@ -44,10 +44,12 @@ int64_t score_select_ctas(int64_t BH, int64_t nQB);
 
 // Step 3, bf16 D=128: TMA + tcgen05 + TMEM kernel (sm_100a), two query blocks
 // per CTA as interleaved pipelines.
+// withhold_kv: a test hook that loads no key or value tile, so that the
+// kernel's first ring wait runs out (SPARSTAR_STATUS_TIMEOUT).
 int launch_attn_sm100(const void *q, const void *k, const void *v, int64_t BH, int64_t Lq,
                       int64_t Lk, float tau, const int32_t *kv_idx, const int32_t *kv_cnt,
                       int64_t max_sel, void *out, float *lse, int32_t *status,
-                      cudaStream_t stream);
+                      cudaStream_t stream, bool withhold_kv = false);
 
 // Step 3, fp32 inputs (D 64/128) and bf16 D=64: fp32 SIMT kernel.
 cudaError_t launch_attn_simt(const void *q, const void *k, const void *v, int dtype,

@@ -56,6 +56,9 @@ def _load():
     L.sparstar_transfer_lists.argtypes = [vp, vp, i64, i64, i64, vp, vp, vp, vp, i64, vp]
     L.sparstar_transfer_max_sel.argtypes = [vp, vp, i64]
     L.sparstar_transfer_max_sel.restype = i64
+    L.sparstar_test_attn_timeout.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, vp, i64, vp, vp,
+                                             vp]
+    L.sparstar_test_attn_timeout.restype = i32
     L.sparstar_strerror.argtypes = [i32]
     L.sparstar_strerror.restype = ctypes.c_char_p
     L.sparstar_version.restype = i32
@@ -389,3 +392,19 @@ def sparstar_transfer_lists(kv_idx, kv_cnt, src_len, dst_len, dst_idx=None, dst_
                                        _ptr(dst_idx), _ptr(dst_cnt), dst_idx.shape[-1],
                                        _stream(stream)), "sparstar_transfer_lists")
     return dst_idx, dst_cnt
+
+
+def sparstar_test_attn_timeout(q, k, v, kv_idx, kv_cnt, out, status, stream=None):
+    """Test hook: the attention kernel with its K/V copies withheld, so that
+    its first ring wait runs out and SPARSTAR_STATUS_TIMEOUT is set in
+    `status` (an int32 device tensor)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _dev(t, n)
+    _dev(kv_idx, "kv_idx", torch.int32)
+    _dev(kv_cnt, "kv_cnt", torch.int32)
+    _dev(status, "status", torch.int32)
+    B, H, Lq, D = q.shape
+    _check(lib.sparstar_test_attn_timeout(_ptr(q), _ptr(k), _ptr(v), B, H, Lq, k.shape[2],
+                                          _ptr(kv_idx), _ptr(kv_cnt), kv_idx.shape[-1],
+                                          _ptr(out), _ptr(status), _stream(stream)),
+           "sparstar_test_attn_timeout")

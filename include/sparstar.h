@@ -369,6 +369,22 @@ int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt, int6
                             int32_t *dst_idx, int32_t *dst_cnt, int64_t dst_max_sel,
                             void *stream);
 
+/*
+ * sparstar_test_attn_timeout — TEST HOOK for failure detection, not part of
+ * the attention forward.  Runs the bf16 D = 128 attention kernel with every
+ * key and value copy withheld: the kernel's first wait on its K/V ring can
+ * never complete, gives up after about two seconds, ORs
+ * SPARSTAR_STATUS_TIMEOUT into *status, and every role leaves through its
+ * abort path (copies in flight drained, TMEM freed), so the CUDA context
+ * stays usable.  `out` is left undefined.  Arguments as for sparstar_attn_fwd
+ * (bf16, D = 128; status required).  Returns a launch status; the timeout is
+ * reported in *status once the stream has run.
+ */
+int sparstar_test_attn_timeout(const void *q, const void *k, const void *v, int64_t B, int64_t H,
+                               int64_t Lq, int64_t Lk, const int32_t *kv_idx,
+                               const int32_t *kv_cnt, int64_t max_sel, void *out,
+                               int32_t *status, void *stream);
+
 /* Message for a status code (static storage). */
 const char *sparstar_strerror(int code);
 
