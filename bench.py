@@ -248,7 +248,7 @@ def run_reference(args, world, rank):
         return
     import oracle as orc
     orc.lib()
-    w = synth.WORKLOADS[args.workload]
+    w = bench_workload(args)
     q, k, v = synth.generate(w)
     qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
     flops = oracle_flops(orc, w, qn, kn)
@@ -279,6 +279,7 @@ def workload_config(w, world):
                         "queries %d, density %g" % (w.name, w.H, w.D, w.dtype, w.text, w.image_ref,
                                                     w.ref, w.cur, w.Lk, w.Lq, w.density),
             "seq_len": w.Lq, "keys": w.Lk, "heads": w.H, "head_dim": w.D, "density": w.density,
+            "seed": w.seed,
             "global_batch": w.B * world, "parallelism": "replicas" if world > 1 else "single",
             "l2": "no flush: inputs (%.2f GB) larger than L2" % (
                 (w.Lq + 2 * w.Lk) * w.H * w.D * (2 if w.dtype == "bf16" else 4) / 1e9)}
@@ -327,7 +328,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.set_device(device)
     from block_sparse_attention_18_b200 import sparstar as sp
 
-    w = synth.WORKLOADS[args.workload]
+    w = bench_workload(args)
     q, k, v = synth.generate(w)
     qd, kd, vd = q.to(device), k.to(device), v.to(device)
     ws = sp.Workspace(w.B, w.H, w.D, w.text, w.image_ref, w.ref, w.cur, w.density, device)
@@ -693,6 +694,13 @@ def dense_comparison(sp, w, qd, kd, vd, tau, sparse_attn_ms, stream, reps=3):
             "speedup_vs_ours_dense": ours / sparse_attn_ms}
 
 
+def bench_workload(args):
+    """The workload named on the command line, with --seed replacing its
+    seed when given (the synthetic inputs are drawn from that seed)."""
+    w = synth.WORKLOADS[args.workload]
+    return w if args.seed is None else synth.with_seed(w, args.seed)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -700,6 +708,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=list(synth.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=None,
+                    help="seed of the synthetic inputs (default: the workload's own)")
     ap.add_argument("--ref-rows", type=int, default=256,
                     help="query rows per sampled step of the reference arm")
     ap.add_argument("--chain", choices=["fused", "separate"], default="fused",

@@ -26,6 +26,7 @@
 #include <mutex>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "sparstar.h"
 #include "sparstar_internal.h"
@@ -67,11 +68,12 @@ size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
 
 }  // namespace
 
-SPARSTAR_API int sparstar_forward_static(const void *q, const void *k, const void *v, int dtype,
-                                         int64_t B, int64_t H, int64_t D, int64_t text_len,
-                                         int64_t image_ref_len, int64_t ref_len, int64_t cur_len,
-                                         double density, void *out, float *lse, int32_t *status,
-                                         void *stream) {
+namespace {
+
+int forward_static_impl(const void *q, const void *k, const void *v, int dtype, int64_t B,
+                        int64_t H, int64_t D, int64_t text_len, int64_t image_ref_len,
+                        int64_t ref_len, int64_t cur_len, double density, void *out, float *lse,
+                        int32_t *status, void *stream) {
     if (B <= 0 || H <= 0 || (D != 64 && D != 128) || text_len < 0 || image_ref_len < 0 ||
         ref_len < 0 || cur_len <= 0)
         return SPARSTAR_EINVAL;
@@ -104,4 +106,18 @@ SPARSTAR_API int sparstar_forward_static(const void *q, const void *k, const voi
     int32_t *kv_cnt = reinterpret_cast<int32_t *>(a + s_qbar + s_kbar + s_S + s_idx);
     return sparstar_forward(q, k, v, dtype, B, H, D, text_len, image_ref_len, ref_len, cur_len,
                             density, qbar, kbar, S, kv_idx, kv_cnt, sel, out, lse, status, stream);
+}
+
+}  // namespace
+
+SPARSTAR_API int sparstar_forward_static(const void *q, const void *k, const void *v, int dtype,
+                                         int64_t B, int64_t H, int64_t D, int64_t text_len,
+                                         int64_t image_ref_len, int64_t ref_len, int64_t cur_len,
+                                         double density, void *out, float *lse, int32_t *status,
+                                         void *stream) {
+    nvtxRangePushA("sparstar_forward_static");  // one NVTX range per ABI call
+    const int rc = forward_static_impl(q, k, v, dtype, B, H, D, text_len, image_ref_len, ref_len,
+                                       cur_len, density, out, lse, status, stream);
+    nvtxRangePop();
+    return rc;
 }

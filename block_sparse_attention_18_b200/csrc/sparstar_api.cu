@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>  // header-only: ranges cost nothing without a tool attached
 
 #include "sparstar.h"
 #include "sparstar_internal.h"
@@ -40,6 +41,15 @@ int device_check() {
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SPARSTAR_OK : SPARSTAR_ECUDA; }
+
+// An NVTX range over one ABI call (host side: argument checks and launches),
+// named after the call, for profilers that group work by NVTX range.
+struct TraceRange {
+    explicit TraceRange(const char *name) { nvtxRangePushA(name); }
+    ~TraceRange() { nvtxRangePop(); }
+    TraceRange(const TraceRange &) = delete;
+    TraceRange &operator=(const TraceRange &) = delete;
+};
 
 // Largest sizes the kernels index with 32-bit grid or coordinate values.
 constexpr int64_t kMaxGrid = 0x7fffffffLL;
@@ -81,6 +91,7 @@ SPARSTAR_API int64_t sparstar_select_count(int64_t nKB, int64_t n_forced_blocks,
 
 SPARSTAR_API int sparstar_block_pool(const void *x, int dtype, int64_t B, int64_t H, int64_t L,
                                      int64_t D, float *xbar, void *stream) {
+    TraceRange trace("sparstar_block_pool");
     if (!dtype_ok(dtype)) return SPARSTAR_EDTYPE;
     if (!x || !xbar || B <= 0 || H <= 0 || L <= 0 || !head_dim_ok(D)) return SPARSTAR_EINVAL;
     if (!aligned16(x) || !aligned16(xbar)) return SPARSTAR_EINVAL;
@@ -93,6 +104,7 @@ SPARSTAR_API int sparstar_block_pool(const void *x, int dtype, int64_t B, int64_
 SPARSTAR_API int sparstar_block_score(const float *qbar, const float *kbar, int64_t B, int64_t H,
                                       int64_t nQB, int64_t nKB, int64_t D, float tau, float *S,
                                       void *stream) {
+    TraceRange trace("sparstar_block_score");
     if (!qbar || !kbar || !S || B <= 0 || H <= 0 || nQB <= 0 || nKB <= 0 || !head_dim_ok(D))
         return SPARSTAR_EINVAL;
     if (!std::isfinite(tau)) return SPARSTAR_EINVAL;
@@ -108,6 +120,7 @@ SPARSTAR_API int sparstar_block_score(const float *qbar, const float *kbar, int6
 SPARSTAR_API int sparstar_select(const float *S, int64_t B, int64_t H, int64_t nQB, int64_t nKB,
                                  int64_t n_forced_blocks, double density, int32_t *kv_idx,
                                  int32_t *kv_cnt, int64_t max_sel, void *stream) {
+    TraceRange trace("sparstar_select");
     if (!S || !kv_idx || !kv_cnt || B <= 0 || H <= 0 || nQB <= 0 || nKB <= 0)
         return SPARSTAR_EINVAL;
     if (nKB > 0x7fffffffLL) return SPARSTAR_EINVAL;
@@ -127,6 +140,7 @@ SPARSTAR_API int sparstar_attn_fwd(const void *q, const void *k, const void *v, 
                                    float tau, const int32_t *kv_idx, const int32_t *kv_cnt,
                                    int64_t max_sel, void *out, float *lse, int32_t *status,
                                    void *stream) {
+    TraceRange trace("sparstar_attn_fwd");
     if (!dtype_ok(dtype)) return SPARSTAR_EDTYPE;
     if (!q || !k || !v || !out || !kv_cnt || B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 ||
         !head_dim_ok(D) || max_sel < 0)
@@ -152,6 +166,7 @@ SPARSTAR_API int sparstar_attn_fwd(const void *q, const void *k, const void *v, 
 SPARSTAR_API int sparstar_block_pool_qk(const void *q, const void *k, int dtype, int64_t B,
                                         int64_t H, int64_t Lq, int64_t Lk, int64_t D,
                                         float *qbar, float *kbar, void *stream) {
+    TraceRange trace("sparstar_block_pool_qk");
     if (!dtype_ok(dtype)) return SPARSTAR_EDTYPE;
     if (!q || !k || !qbar || !kbar || B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 ||
         !head_dim_ok(D))
@@ -176,6 +191,7 @@ SPARSTAR_API int sparstar_score_select(const float *qbar, const float *kbar, int
                                        int64_t n_forced_blocks, double density, int32_t *kv_idx,
                                        int32_t *kv_cnt, int64_t max_sel, int32_t *status,
                                        void *stream) {
+    TraceRange trace("sparstar_score_select");
     if (!qbar || !kbar || !kv_idx || !kv_cnt || B <= 0 || H <= 0 || nQB <= 0 || nKB <= 0 ||
         !head_dim_ok(D))
         return SPARSTAR_EINVAL;
@@ -198,6 +214,7 @@ SPARSTAR_API int sparstar_forward(const void *q, const void *k, const void *v, i
                                   double density, float *qbar, float *kbar, float *S,
                                   int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel, void *out,
                                   float *lse, int32_t *status, void *stream) {
+    TraceRange trace("sparstar_forward");
     if (text_len < 0 || image_ref_len < 0 || ref_len < 0 || cur_len <= 0 || !head_dim_ok(D))
         return SPARSTAR_EINVAL;
     const int64_t Lq = cur_len, Lk = text_len + image_ref_len + ref_len + cur_len;
@@ -224,6 +241,7 @@ SPARSTAR_API int sparstar_forward_fused(const void *q, const void *k, const void
                                         double density, float *qbar, float *kbar,
                                         int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel,
                                         void *out, float *lse, int32_t *status, void *stream) {
+    TraceRange trace("sparstar_forward_fused");
     if (text_len < 0 || image_ref_len < 0 || ref_len < 0 || cur_len <= 0 || !head_dim_ok(D))
         return SPARSTAR_EINVAL;
     const int64_t Lq = cur_len, Lk = text_len + image_ref_len + ref_len + cur_len;
@@ -250,6 +268,7 @@ SPARSTAR_API int sparstar_retained_mass(const void *q, const void *k, int dtype,
                                         const int64_t *rows, int64_t n_rows, float *scratch,
                                         double *lse_dense, double *mass_block, double *mass_tok,
                                         double *mass_forced, void *stream) {
+    TraceRange trace("sparstar_retained_mass");
     if (!dtype_ok(dtype)) return SPARSTAR_EDTYPE;
     if (!q || !k || !kv_cnt || !rows || !scratch || !lse_dense || !mass_block || !mass_tok ||
         !mass_forced || B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 || !head_dim_ok(D) ||
@@ -307,6 +326,7 @@ SPARSTAR_API int sparstar_transfer_lists(const int32_t *src_idx, const int32_t *
                                          const int64_t *src_len, const int64_t *dst_len,
                                          int32_t *dst_idx, int32_t *dst_cnt, int64_t dst_max_sel,
                                          void *stream) {
+    TraceRange trace("sparstar_transfer_lists");
     if (!src_idx || !src_cnt || !dst_idx || !dst_cnt || B <= 0 || H <= 0 ||
         dst_max_sel > 0x7fffffffLL)
         return SPARSTAR_EINVAL;
@@ -331,6 +351,7 @@ SPARSTAR_API int sparstar_test_attn_timeout(const void *q, const void *k, const 
                                             const int32_t *kv_idx, const int32_t *kv_cnt,
                                             int64_t max_sel, void *out, int32_t *status,
                                             void *stream) {
+    TraceRange trace("sparstar_test_attn_timeout");
     if (!q || !k || !v || !out || !kv_cnt || !status || B <= 0 || H <= 0 || Lq <= 0 ||
         Lk <= 0 || max_sel < 0 || (max_sel > 0 && !kv_idx))
         return SPARSTAR_EINVAL;
