@@ -698,7 +698,8 @@ def bench_workload(args):
     """The workload named on the command line, with --seed replacing its
     seed when given (the synthetic inputs are drawn from that seed)."""
     w = synth.WORKLOADS[args.workload]
-    return w if args.seed is None else synth.with_seed(w, args.seed)
+    seed = getattr(args, "seed", None)
+    return w if seed is None else synth.with_seed(w, seed)
 
 
 def main(argv=None):
