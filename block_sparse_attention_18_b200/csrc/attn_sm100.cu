@@ -425,14 +425,26 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int x = 0; x < 2; ++x) {
             const int32_t *lx = x ? listB : listA;
             const int cx = x ? cntB : cntA;
+            // Four loads in flight per lane: the entries are independent, and
+            // this count is on the path from the CTA's start to its first S.
             int nv = 0;
-            for (int c = lane; c < cx; c += 32) {
-                const int j = __ldg(lx + c);
-                if (j >= 0 && j < nKB)
-                    ++nv;
-                else if (status)
-                    atomicOr(status, SPARSTAR_STATUS_BAD_INDEX);
+            bool bad = false;
+            int c = lane;
+            for (; c + 96 < cx; c += 128) {
+                const int j0 = __ldg(lx + c), j1 = __ldg(lx + c + 32);
+                const int j2 = __ldg(lx + c + 64), j3 = __ldg(lx + c + 96);
+                const bool v0 = j0 >= 0 && j0 < nKB, v1 = j1 >= 0 && j1 < nKB;
+                const bool v2 = j2 >= 0 && j2 < nKB, v3 = j3 >= 0 && j3 < nKB;
+                nv += (int)v0 + (int)v1 + (int)v2 + (int)v3;
+                bad |= !(v0 && v1 && v2 && v3);
             }
+            for (; c < cx; c += 32) {
+                const int j = __ldg(lx + c);
+                const bool v = j >= 0 && j < nKB;
+                nv += (int)v;
+                bad |= !v;
+            }
+            if (bad && status) atomicOr(status, SPARSTAR_STATUS_BAD_INDEX);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, o);
             if (lane == 0) bars->n_valid[x] = nv;
