@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # SHA-256 of the kernel source it was taken on; reported only while the
 # source is unchanged.
 ATTN_TRAFFIC = {
-    "source_sha256": "9facb2a518e673ec263dd412ce884f1893d7e3cf17d640e676bc4d24d368f8ed",
-    "bytes_per_launch": 3576933888 + 297030400,  # largest workload, one launch
+    "source_sha256": "86fc765e3339fad23cbae11967a36cb4492735509520144ab9235526a8213179",
+    "bytes_per_launch": 3505765888 + 292825344,  # largest workload, one launch
 }
 
 
