@@ -167,9 +167,7 @@ int sparstar_select(const float *S, int64_t B, int64_t H, int64_t nQB, int64_t n
  * list is empty gets out = 0 and lse = -inf.  bf16 with D = 128 runs on the
  * tcgen05 tensor-core kernel (fp32 accumulation and softmax, P rounded to
  * bf16 for the second product); fp32 inputs and D = 64 run on an fp32 SIMT
- * kernel.  The tensor-core kernel returns SPARSTAR_ESIZE, launching
- * nothing, for more than 65,535 key blocks (Lk above 8,388,480) or more
- * than 2^31 - 1 pairs of query blocks (B * H * ceil(nQB / 2)).
+ * kernel.
  */
 int sparstar_attn_fwd(const void *q, const void *k, const void *v, int dtype, int64_t B,
                       int64_t H, int64_t Lq, int64_t Lk, int64_t D, float tau,

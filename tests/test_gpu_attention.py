@@ -156,3 +156,28 @@ def test_every_list_length_pair_up_to_12(sp, orc):
             cnt[0, h, i] = n
     rows = parity.sample_rows(w.B, w.H, w.Lq, per_head_blocks=18, rows_per_block=4, seed=5)
     _run(sp, orc, w, idx=idx, cnt=cnt, rows=rows)
+
+
+def test_many_pairs_with_uneven_lists(sp, orc):
+    """More query-block pairs than SMs (16 heads x 24 pairs = 384), each
+    block with a random list length in 0..7: pairs where one block has
+    several more tiles than the other (a run of one block's P hand-offs at
+    the end of the pair), blocks without tiles beside blocks with tiles, and
+    consecutive pairs of a head with different mixes."""
+    w = synth.custom(H=16, D=128, dtype="bf16", text=128, ref=1024, cur=48 * 128,
+                     density=1.0, seed=91)
+    nQB, nKB = w.nQB, w.nKB
+    assert nQB == 48 and nKB >= 8
+    rng = np.random.default_rng(4)
+    idx = np.full((1, w.H, nQB, 7), -1, np.int32)
+    cnt = np.zeros((1, w.H, nQB), np.int32)
+    for h in range(w.H):
+        for i in range(nQB):
+            n = int(rng.integers(0, 8))
+            idx[0, h, i, :n] = np.sort(rng.choice(nKB, size=n, replace=False))
+            cnt[0, h, i] = n
+    # uneven pairs (one block at least two tiles longer) are common
+    pairs = cnt.reshape(w.H, nQB // 2, 2)
+    assert (np.abs(pairs[..., 0] - pairs[..., 1]) >= 2).sum() > 100
+    rows = parity.sample_rows(w.B, w.H, w.Lq, per_head_blocks=48, rows_per_block=2, seed=6)
+    _run(sp, orc, w, idx=idx, cnt=cnt, rows=rows)
