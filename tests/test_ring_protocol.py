@@ -131,3 +131,41 @@ def test_one_full_barrier_per_stage_would_not_be_exact():
               if any(e - STAGES >= 0 and e - STAGES not in landed
                      for e, landed in landed_before_tests(nA, nB))]
     assert (2, 3) in unsafe  # PV(A, 1) tests slot 7 while K(B, 1) (slot 3) may be in flight
+
+
+def hand_off_order(nA, nB):
+    """The P hand-offs of one pair in the kernel's order: A(0), B(0), A(1),
+    B(1), ... (a block past its last tile drops out)."""
+    return [(x, j) for j in range(max(nA, nB)) for x in range(2) if j < (nA, nB)[x]]
+
+
+def previous_hand_off(x, j, nA, nB):
+    """The hand-off whose O += P V the softmax of block x waits for before
+    storing P of its tile j, as the kernel computes it (None for the first)."""
+    if x == 0:
+        return None if j < 1 else ((1, j - 1) if j - 1 < nB else (0, j - 1))
+    if j < nA:
+        return (0, j)
+    return (1, j - 1) if j >= 1 else None
+
+
+@pytest.mark.parametrize("nA", range(0, 13))
+def test_hand_off_waits_are_exact_within_a_pair(nA):
+    """Block x tests, by parity, the phase of the previous hand-off (block
+    y, its k-th) on y's barrier.  The test is exact when y's phase k - 1 is
+    complete; x knows every hand-off before its own previous one complete
+    (it waited for the one just before that, and the MMAs complete in
+    issue order)."""
+    for nB in range(0, 13):
+        order = hand_off_order(nA, nB)
+        pos = {h: m for m, h in enumerate(order)}
+        last_own = {}
+        for m, (x, j) in enumerate(order):
+            prev = previous_hand_off(x, j, nA, nB)
+            assert prev == (order[m - 1] if m else None)  # the chain's predecessor
+            if prev is not None:
+                y, k = prev
+                if k >= 1:
+                    known = last_own.get(x, -1) - 1
+                    assert pos[(y, k - 1)] <= known, (nA, nB, x, j)
+            last_own[x] = m
