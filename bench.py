@@ -78,7 +78,7 @@ def attention_flops(kv_idx: np.ndarray, kv_cnt: np.ndarray, Lq: int, Lk: int, D:
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons every 50 ms while
+    """Samples nvidia-smi clocks and throttle reasons every 20 ms while
     running.  Each sample keeps its host arrival time, so that summary()
     can keep only the samples taken inside a given window (the timed
     region); started ahead of the region, it is already sampling when the
@@ -105,7 +105,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self._gpu_id(), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
