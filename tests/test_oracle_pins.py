@@ -251,6 +251,91 @@ def test_fp32_selection_agrees_with_fp64_off_near_ties(orc):
     assert not np.any(differ & ~near)
 
 
+# The near-tie rule: with a row's candidate scores sorted descending
+# s(1) >= s(2) >= ..., the row's gap is s(k) - s(k+1) and its scale is the
+# largest |S| over the candidates (forced blocks are not ranked, so they take
+# no part).  Each row below is built so that its gap and scale are known
+# without sorting anything.
+
+def _gaps(orc, rows, nF, k):
+    S = np.array(rows, np.float64)
+    return orc.near_tie_gaps(S, nF, k)
+
+
+def test_near_tie_gap_hand_built_rows(orc):
+    # nF = 2 forced blocks hold the row's largest |S| (-200, 100): they must
+    # not enter the scale.  Candidates (after the forced prefix):
+    #   row 0: 3, 1, 7, 5     -> descending 7 5 | 3 1      gap 5 - 3 = 2, scale 7
+    #   row 1: 4, 2, 4, 1     -> descending 4 4 | 2 1      gap 4 - 2 = 2, scale 4
+    #   row 2: -3, -1, -7, -2 -> descending -1 -2 | -3 -7  gap 1, scale 7
+    #   row 3: 9, 4.5, 10, 5  -> descending 10 9 | 5 4.5   gap 4 (the steps
+    #          before and after it are 1 and 0.5, so an index off by one
+    #          on either side gives another value)
+    rows = [[100.0, -200.0, 3.0, 1.0, 7.0, 5.0],
+            [-200.0, 100.0, 4.0, 2.0, 4.0, 1.0],
+            [100.0, -200.0, -3.0, -1.0, -7.0, -2.0],
+            [-200.0, 100.0, 9.0, 4.5, 10.0, 5.0]]
+    gap, scale = _gaps(orc, rows, 2, 2)
+    assert gap.tolist() == [2.0, 2.0, 1.0, 4.0]
+    assert scale.tolist() == [7.0, 4.0, 7.0, 10.0]
+
+
+def test_near_tie_gap_exact_tie_at_the_boundary(orc):
+    # k = 1 with two equal leaders: s(1) = s(2) = 4, gap exactly 0.
+    gap, scale = _gaps(orc, [[9.0, 2.0, 4.0, 1.0, 4.0]], 1, 1)
+    assert gap[0] == 0.0 and scale[0] == 4.0
+    # k = 2 on the same row: descending 4 4 | 2 1, gap 2.
+    gap, _ = _gaps(orc, [[9.0, 2.0, 4.0, 1.0, 4.0]], 1, 2)
+    assert gap[0] == 2.0
+
+
+def test_near_tie_gap_is_infinite_when_nothing_or_everything_is_kept(orc):
+    rows = [[5.0, 3.0, 1.0, 2.0], [0.0, -1.0, -1.0, -1.0]]
+    for k in (0, 3):  # C = 3 candidates after nF = 1
+        gap, scale = _gaps(orc, rows, 1, k)
+        assert np.all(np.isposinf(gap))
+        assert scale.tolist() == [3.0, 1.0]
+
+
+def test_near_tie_gap_on_shuffled_rows_with_distinct_steps(orc):
+    # Each row is a shuffle of v_1 > v_2 > ... whose steps v_i - v_{i+1}
+    # are distinct powers of two (exact in fp64), so the gap at k is the
+    # k-th step and nothing else; the rows differ, which also pins the row
+    # stride.  Forced blocks carry values far outside the candidates.
+    rng = np.random.default_rng(7)
+    C, nF, nrow = 11, 3, 6
+    rows, want_gap, want_scale = [], {}, []
+    for r in range(nrow):
+        steps = [2.0 ** e for e in rng.permutation(C - 1)]
+        top = float(rng.integers(-40, 40))
+        vals = [top]
+        for s in steps:
+            vals.append(vals[-1] - s)
+        want_scale.append(max(abs(vals[0]), abs(vals[-1])))
+        for k in range(1, C):
+            want_gap[(r, k)] = steps[k - 1]
+        forced = [1e6 * (1 + r), -2e6, 3e6]
+        rows.append(forced + [vals[i] for i in rng.permutation(C)])
+    for k in range(1, C):
+        gap, scale = _gaps(orc, rows, nF, k)
+        assert gap.tolist() == [want_gap[(r, k)] for r in range(nrow)], k
+        assert scale.tolist() == want_scale
+
+
+def test_near_tie_rule_flags_exactly_the_close_rows(orc):
+    # The decision the GPU tests take from these values: gap < 1e-6 * scale.
+    # Candidates 0.5, 0.5 - d, 0.25 with k = 1, so the scale is 0.5.
+    # Row 0: d = 1e-7 -> near.  Row 1: d = 1e-5 -> not near.
+    # Row 2: an exact tie -> near.  Row 3: k = C -> never near.
+    rows = [[1.0, 0.5, 0.5 - 1e-7, 0.25], [1.0, 0.5, 0.5 - 1e-5, 0.25],
+            [1.0, 0.5, 0.5, 0.25]]
+    gap, scale = _gaps(orc, rows, 1, 1)
+    near = gap < 1e-6 * scale
+    assert near.tolist() == [True, False, True]
+    gap, scale = _gaps(orc, rows, 1, 3)
+    assert not np.any(gap < 1e-6 * scale)
+
+
 # ------------------------------------------------------------- attention
 
 def _to_f64(x):
