@@ -6,26 +6,28 @@
 // One CTA per (b, h, pair of query blocks 2p, 2p+1), head-major, so the CTAs
 // that run together share one head's K/V in L2.  The two query blocks, A
 // and B, have their own block lists and run as two interleaved pipelines:
-// while the softmax of one works, the tensor core multiplies for the other,
-// and the two softmax warpgroups drift half a period apart so their
-// exponentials (MUFU) and their TMEM traffic overlap.  Eleven warps:
+// while the softmax of one works, the tensor core multiplies for the other.
+// Eleven warps:
 //   warps 0-3  softmax + epilogue of block A, warps 4-7 of block B: warp w
 //              serves TMEM lanes 32*(w%4)..+31, one query row per thread,
 //              all 128 columns of each key tile;
-//   warp 8     TMA producer: Q_A and Q_B once, then K(0), K(1), V(0),
-//              K(2), V(1), ... (each for A and B) through a 4-stage ring;
-//   warp 9     TMEM allocation and the S = Q K^T MMAs (A then B per step);
-//   warp 10    the O += P V MMAs (A then B per step).
-// TMEM (512 columns): S_A at 0, S_B at 128 (fp32 128 x 128), O_A at 256,
-// O_B at 384.  The softmax frees S_X as soon as it has read it into
-// registers, so S_X(j+1) = Q_X K(j+1)^T runs on the tensor core while the
-// softmax of tile j computes its exponentials.  P (bf16) goes to shared
-// memory as the K-major, 128-byte-swizzled A operand of O_X += P V; A and B
-// hand their P tiles over through one buffer in turn, each hand-off waiting
-// for the O += P V of the one before it (on that block's completion
-// barrier, so every parity wait targets the current or the next phase).
-// Shared memory: Q_A, Q_B, P (32 KB each) and a 4-stage K/V ring whose
-// keys run two steps ahead of its values.
+//   warp 8     TMA producer: Q_A and Q_B once, then the key and value tiles
+//              through a 5-stage ring in the order the MMAs consume them:
+//              K_A(0), K_B(0), then per step j: K_A(j+1), V_A(j), K_B(j+1),
+//              V_B(j);
+//   warp 9     TMEM allocation and the S = Q K^T MMAs, in the order A(0),
+//              B(0), A(1), B(1), ...;
+//   warp 10    the O += P V MMAs, in the same order.
+// TMEM (512 columns): one S buffer at 0 (fp32 128 x 128) that the two blocks
+// take in turn, P_A at 128 and P_B at 192 (bf16, two per column), O_A at
+// 256 and O_B at 384.  The softmax of a block frees S as soon as it has read
+// its scores into registers, so the other block's S = Q K^T runs on the
+// tensor core while this one computes its exponentials.  P goes to tensor
+// memory with tcgen05.st and is the A operand of O += P V (tcgen05.mma with
+// A in tensor memory, B = V from shared memory), handed over in two 64-key
+// halves so that the first half's MMAs start while the second half's
+// exponentials run.  P never touches shared memory, which holds only Q_A,
+// Q_B and the ring.
 //
 // Each row runs an online softmax in log2 units (running max m, sum l,
 // accumulator O_X in TMEM); O_X and l are rescaled only when the tile max
@@ -47,36 +49,37 @@ namespace sparstar {
 namespace {
 
 constexpr int kHD = 128;                      // head dim
-constexpr int kStages = 4;                    // K/V ring depth
+constexpr int kStages = 5;                    // K/V ring depth
 constexpr int kTileBytes = kBlock * kHD * 2;  // 32 KB: one Q, K or V tile
 constexpr int kPanelBytes = kTileBytes / 2;   // 16 KB: 128 rows x 64 columns
 constexpr int kSoftmaxThreads = 256;          // warps 0-7 (128 per query block)
 constexpr int kThreads = kSoftmaxThreads + 96;
 constexpr int kProducerWarp = 8, kMmaWarp = 9, kPvWarp = 10;
 constexpr uint32_t kTmemCols = 512;
-__host__ __device__ constexpr uint32_t col_s(int x) { return x ? 128u : 0u; }  // S_A, S_B
+constexpr uint32_t kColS = 0;                                                    // S (A and B in turn)
+__host__ __device__ constexpr uint32_t col_p(int x) { return x ? 192u : 128u; }  // P_A, P_B
 __host__ __device__ constexpr uint32_t col_o(int x) { return x ? 384u : 256u; }  // O_A, O_B
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
 constexpr int kOffQ = 0;                          // Q_A, then Q_B
-constexpr int kOffP = 2 * kTileBytes;             // P (bf16, K-major, swizzled), A and B in turn
-constexpr int kOffStage = 3 * kTileBytes;
+constexpr int kOffStage = 2 * kTileBytes;
 constexpr int kOffBar = kOffStage + kStages * kTileBytes;
 struct Bars {
     uint64_t q_full;
     uint64_t st_full[kStages][2];  // [stage][use & 1]
     uint64_t st_empty[kStages];
-    uint64_t s_full[2];   // per query block
-    uint64_t s_free[2];
-    uint64_t p_full[2][2];   // [block][half of P]: keys 64h .. 64h+63 written
-    uint64_t pv_half[2][2];  // [block][half]: O += P_half V_half complete
+    uint64_t s_full[2];      // per query block: S holds this block's scores
+    uint64_t s_free;         // the reader of the latest S has it in registers
+    uint64_t p_full[2][2];   // [block][half of P]: keys 64h .. 64h+63 stored
+    uint64_t pv_done[2];     // per block: O += P V complete (P buffer free)
     uint64_t drain;
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t n_valid[2];
 };
 constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, M = N = 128.
 constexpr uint32_t make_idesc(bool b_mn_major) {
@@ -235,6 +238,15 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// A in tensor memory (P), B from shared memory (V).
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -254,6 +266,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "%28, %29, %30, %31}, [%32];"
         : SPX_R8(0), SPX_R8(8), SPX_R8(16), SPX_R8(24)
         : "r"(taddr));
+}
+// 32 consecutive 32-bit columns of this thread's TMEM lane from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+        "%27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        SPX_W8(0), SPX_W8(8), SPX_W8(16), SPX_W8(24)
+        : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -324,21 +345,28 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                  : "memory");
 }
 
-// Producer order: K(0), K(1), then for s = 0, 1, ...: V(s), K(s+2), where
-// K(j) stands for K_A(j), K_B(j) and V(j) for V_A(j), V_B(j), each present
-// while j is below that block's tile count.  Keys run two steps ahead of
-// values, so the next S products never wait for a value tile's slot.
-// C(m) counts the tiles of steps before m; the ring index of each tile is
-// the number of tiles the producer loads before it.
-__device__ __forceinline__ int steps_before(int m, int nA, int nB) {
-    m = m < 0 ? 0 : m;
-    return (m < nA ? m : nA) + (m < nB ? m : nB);
+// Producer order (the order the MMA warps consume the tiles): K(A,0),
+// K(B,0), then for j = 0, 1, ...: K(A,j+1), V(A,j), K(B,j+1), V(B,j), each
+// present while its tile index is below that block's tile count.  The ring
+// index of a tile is the number of tiles loaded before it; loads_before(j)
+// counts the tiles ahead of step j's group.
+__device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
+__device__ __forceinline__ int loads_before(int j, int nA, int nB) {
+    int c = (nA > 0) + (nB > 0);
+    c += imin(j, nA - 1) > 0 ? imin(j, nA - 1) : 0;
+    c += imin(j, nA);
+    c += imin(j, nB - 1) > 0 ? imin(j, nB - 1) : 0;
+    c += imin(j, nB);
+    return c;
 }
 __device__ __forceinline__ int slot_k(int x, int j, int nA, int nB) {
-    return steps_before(j, nA, nB) + steps_before(j - 1, nA, nB) + ((x == 1 && j < nA) ? 1 : 0);
+    if (j == 0) return x == 0 ? 0 : (nA > 0 ? 1 : 0);
+    const int g = j - 1, b = loads_before(g, nA, nB);
+    return x == 0 ? b : b + (g + 1 < nA) + (g < nA);
 }
 __device__ __forceinline__ int slot_v(int x, int j, int nA, int nB) {
-    return steps_before(j + 2, nA, nB) + steps_before(j, nA, nB) + ((x == 1 && j < nA) ? 1 : 0);
+    const int b = loads_before(j, nA, nB);
+    return x == 0 ? b + (j + 1 < nA) : b + (j + 1 < nA) + (j < nA) + (j + 1 < nB);
 }
 // The QK warp consumes the key tiles and the PV warp the value tiles, so a
 // stage's previous occupant (slot e - kStages) can be the other warp's tile
@@ -384,17 +412,15 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 
     const uint32_t bar_q = smem_addr(&bars->q_full);
     // Ring slot e is use e / kStages of stage e % kStages; each stage has two
-    // full barriers that alternate between its uses (see ring_wait).
+    // full barriers that alternate between its uses (see ring_parity).
     auto bar_full = [&](int e) {
         return smem_addr(&bars->st_full[e % kStages][(e / kStages) & 1]);
     };
     auto bar_empty = [&](int s) { return smem_addr(&bars->st_empty[s]); };
     auto bar_s = [&](int x) { return smem_addr(&bars->s_full[x]); };
-    auto bar_sfree = [&](int x) { return smem_addr(&bars->s_free[x]); };
+    const uint32_t bar_sfree = smem_addr(&bars->s_free);
     auto bar_p = [&](int x, int h) { return smem_addr(&bars->p_full[x][h]); };
-    auto bar_ph = [&](int x, int h) { return smem_addr(&bars->pv_half[x][h]); };
-    // the whole O += P V of a block (its second half completes last)
-    auto bar_pv = [&](int x) { return smem_addr(&bars->pv_half[x][1]); };
+    auto bar_pv = [&](int x) { return smem_addr(&bars->pv_done[x]); };
     const uint32_t bar_drain = smem_addr(&bars->drain);
 
     // ---- set-up: barriers, valid-entry counts, TMEM
@@ -406,13 +432,11 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 mbar_init(smem_addr(&bars->st_full[s][1]), 1);
                 mbar_init(bar_empty(s), 1);
             }
+            mbar_init(bar_sfree, kSoftmaxThreads / 2);  // one block's softmax threads
             for (int x = 0; x < 2; ++x) {
                 mbar_init(bar_s(x), 1);
-                mbar_init(bar_sfree(x), kSoftmaxThreads / 2);
-                for (int h = 0; h < 2; ++h) {
-                    mbar_init(bar_p(x, h), kSoftmaxThreads / 2);
-                    mbar_init(bar_ph(x, h), 1);
-                }
+                for (int h = 0; h < 2; ++h) mbar_init(bar_p(x, h), kSoftmaxThreads / 2);
+                mbar_init(bar_pv(x), 1);
             }
             mbar_init(bar_drain, 2);  // one commit from each MMA warp
             bars->abort_flag = 0;
@@ -477,35 +501,38 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             int curKA = 0, curKB = 0, curVA = 0, curVB = 0;
             int e = 0;
-            bool ok = true;
-            // Groups K(0), K(1), V(0), K(2), V(1), K(3), ...: group g > 0
-            // is K((g+1)/2) when odd, V(g/2-1) when even.
             // withhold_kv (a test hook): no key or value tile is loaded, so
             // the first wait on the ring runs out and every role takes its
             // abort path.
-            for (int g = 0; g <= 2 * nmax && ok && !withhold_kv; ++g) {
-                const bool is_v = g > 0 && (g & 1) == 0;
-                const int j = g == 0 ? 0 : (is_v ? g / 2 - 1 : (g + 1) / 2);
-                for (int x = 0; x < 2 && ok; ++x) {
-                    if (j >= (x == 0 ? nA : nB)) continue;
-                    const int stage = e % kStages;
-                    if (!wait1(bar_empty(stage), ((uint32_t)(e / kStages) & 1u) ^ 1u, abort_flag,
-                               status)) {
-                        ok = false;
-                        break;
-                    }
-                    const int32_t *lx = x ? listB : listA;
-                    const int cx = x ? cntB : cntA;
-                    int &cr = is_v ? (x ? curVB : curVA) : (x ? curKB : curKA);
-                    const int kb = next_valid(lx, cx, cr, nKB);
-                    const uint32_t dst = base + kOffStage + stage * kTileBytes;
-                    const CUtensorMap *map = is_v ? &tmV : &tmK;
-                    mbar_expect_tx(bar_full(e), kTileBytes);
-                    tma_load_3d(dst, map, bar_full(e), 0, kb * kBlock, bh, pol_kv);
-                    tma_load_3d(dst + kPanelBytes, map, bar_full(e), 64, kb * kBlock, bh,
-                                pol_kv);
-                    ++e;
+            bool ok = !withhold_kv;
+            // The next key (is_v false) or value tile of block x into ring
+            // slot e.
+            auto load = [&](bool is_v, int x) {
+                if (!ok) return;
+                const int stage = e % kStages;
+                if (!wait1(bar_empty(stage), ((uint32_t)(e / kStages) & 1u) ^ 1u, abort_flag,
+                           status)) {
+                    ok = false;
+                    return;
                 }
+                const int32_t *lx = x ? listB : listA;
+                const int cx = x ? cntB : cntA;
+                int &cr = is_v ? (x ? curVB : curVA) : (x ? curKB : curKA);
+                const int kb = next_valid(lx, cx, cr, nKB);
+                const uint32_t dst = base + kOffStage + stage * kTileBytes;
+                const CUtensorMap *map = is_v ? &tmV : &tmK;
+                mbar_expect_tx(bar_full(e), kTileBytes);
+                tma_load_3d(dst, map, bar_full(e), 0, kb * kBlock, bh, pol_kv);
+                tma_load_3d(dst + kPanelBytes, map, bar_full(e), 64, kb * kBlock, bh, pol_kv);
+                ++e;
+            };
+            if (nA > 0) load(false, 0);
+            if (nB > 0) load(false, 1);
+            for (int j = 0; j < nmax && ok; ++j) {
+                if (j + 1 < nA) load(false, 0);
+                if (j < nA) load(true, 0);
+                if (j + 1 < nB) load(false, 1);
+                if (j < nB) load(true, 1);
             }
             // Copies in flight must land before the CTA may exit: wait for
             // Q and for the latest arming of every stage (no-ops normally).
@@ -518,9 +545,12 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         // -------------------------------------------- S = Q K^T MMA issuer
         // Warp-uniform control flow; one elected lane issues.  Descriptors
         // are built once per operand and advanced by compile-time offsets.
+        // The n-th product (order A(0), B(0), A(1), ...) overwrites S once
+        // the reader of product n - 1 has its scores in registers.
         const uint64_t dQ0 = desc_k_major(base + kOffQ);
         const uint64_t dQ1 = desc_k_major(base + kOffQ + kTileBytes);
         bool ok = nmax > 0 && wait_warp(bar_q, 0, abort_flag, status);
+        int n = 0;
         for (int j = 0; j < nmax && ok; ++j) {
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
@@ -531,9 +561,8 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     ok = false;
                     break;
                 }
-                if (j >= 1) {
-                    // S_x is free once the softmax has read S_x(j-1).
-                    if (!wait_warp(bar_sfree(x), (uint32_t)(j - 1) & 1u, abort_flag, status)) {
+                if (n >= 1) {
+                    if (!wait_warp(bar_sfree, (uint32_t)(n - 1) & 1u, abort_flag, status)) {
                         ok = false;
                         break;
                     }
@@ -541,18 +570,18 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
                 const uint64_t dK = desc_k_major(base + kOffStage + stage * kTileBytes);
                 const uint64_t dQ = x == 0 ? dQ0 : dQ1;
-                const uint32_t dS = tmem + col_s(x);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < kHD / 16; ++kk) {
                         const uint64_t off =
                             (uint64_t)(((kk >> 2) * kPanelBytes + (kk & 3) * 32) >> 4);
-                        mma_ss(dS, dQ + off, dK + off, kIdescQK, kk > 0 ? 1u : 0u);
+                        mma_ss(tmem + kColS, dQ + off, dK + off, kIdescQK, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar_empty(stage));
                     mma_commit(bar_s(x));
                 }
                 __syncwarp();
+                ++n;
             }
         }
         // Drain: every MMA this warp issued completes before TMEM is freed.
@@ -562,6 +591,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
     } else if (warp == kPvWarp) {
         // ---------------------------------------------- O += P V MMA issuer
+        // A = P_x in tensor memory (8 columns per K = 16 step), B = V.
         bool ok = nmax > 0;
         for (int j = 0; j < nmax && ok; ++j) {
 #pragma unroll
@@ -571,7 +601,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     ok = false;
                     break;
                 }
-                tc_fence_after();  // orders an O rescale (tcgen05.st) before the MMA
+                tc_fence_after();  // orders the softmax's tcgen05.st (P, O rescale) first
                 const int e = slot_v(x, j, nA, nB);
                 const int stage = e % kStages;
                 if (!wait_warp(bar_full(e), ring_parity(e), abort_flag, status)) {
@@ -579,26 +609,31 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                     break;
                 }
                 const uint64_t dV = desc_mn_major(base + kOffStage + stage * kTileBytes);
-                const uint64_t dP = desc_k_major(base + kOffP);
+                const uint32_t aP = tmem + col_p(x);
                 const uint32_t first = j > 0 ? 1u : 0u;
-                // Each half of P (keys 64h .. 64h+63, one 16 KB panel) is
-                // multiplied as soon as it is written.
+                // Each half of P (keys 64h .. 64h+63, columns 32h .. 32h+31)
+                // is multiplied as soon as it is stored.
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    if (h == 1 && !wait_warp(bar_p(x, 1), (uint32_t)j & 1u, abort_flag, status)) {
-                        ok = false;
-                        break;
+                    if (h == 1) {
+                        if (!wait_warp(bar_p(x, 1), (uint32_t)j & 1u, abort_flag, status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
                     }
                     if (elect_one()) {
 #pragma unroll
                         for (int kq = 0; kq < 4; ++kq) {
                             const int kk = 4 * h + kq;
-                            mma_ss(tmem + col_o(x), dP + (uint64_t)((h * kPanelBytes + kq * 32) >> 4),
+                            mma_ts(tmem + col_o(x), aP + 8u * kk,
                                    dV + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV,
                                    kk > 0 ? 1u : first);
                         }
-                        if (h == 1) mma_commit(bar_empty(stage));
-                        mma_commit(bar_ph(x, h));
+                        if (h == 1) {
+                            mma_commit(bar_empty(stage));
+                            mma_commit(bar_pv(x));
+                        }
                     }
                     __syncwarp();
                 }
@@ -618,7 +653,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int quarter = warp & 3;      // TMEM lane quarter
         const int row = quarter * 32 + lane;  // TMEM lane == tile row
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const uint32_t colS = col_s(x), colO = col_o(x);
+        const uint32_t colO = col_o(x), colP = col_p(x);
         const int nx = x == 0 ? nA : nB;
         const float sc = tau * 1.4426950408889634f;  // scores in log2 units
         float m_ref = -INFINITY, l = 0.0f;
@@ -640,7 +675,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             {
                 uint32_t r[4][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + colS + 32 * c, r[c]);
+                for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + kColS + 32 * c, r[c]);
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) reg_fence(r[c]);
@@ -649,9 +684,10 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
                     for (int u = 0; u < 32; ++u) s[32 * c + u] = __uint_as_float(r[c][u]);
             }
-            // S_x(j) is in registers: the next S = Q K^T may overwrite it.
+            // The scores are in registers: the other block's S = Q K^T may
+            // overwrite S.
             tc_fence_before();
-            mbar_arrive(bar_sfree(x));
+            mbar_arrive(bar_sfree);
             const int valid = Lk - kb * kBlock;  // keys of this tile that exist
             if (has_tail && valid < kBlock) {
 #pragma unroll
@@ -670,7 +706,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             for (int t = 0; t < 4; ++t) mx[t] = fmaxf(mx[t], s[kBlock - 4 + t]);
             const float m_tile = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sc;
             const float m_new = fmaxf(m_ref, m_tile);
-            bool p_free = false;  // the P buffer is free for this hand-off
+            bool pv_seen = false;  // the O += P V of tile j - 1 is known complete
             if (__any_sync(0xffffffffu, m_new > m_ref + 8.0f)) {
                 if (j > 0) {
                     if (!wait_warp(bar_pv(x), (uint32_t)(j - 1) & 1u, abort_flag, status)) {
@@ -678,6 +714,7 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                         break;
                     }
                     tc_fence_after();
+                    pv_seen = true;
                     const float f = m_new > -INFINITY ? ex2(m_ref - m_new) : 1.0f;
 #pragma unroll 1
                     for (int c = 0; c < kHD / 8; ++c) {
@@ -701,73 +738,48 @@ attn_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             // m_ref = -inf only while every key so far was masked: then
             // every p is 0 (a finite offset keeps -inf * sc + offset = -inf).
             const float neg_m = m_ref > -INFINITY ? -m_ref : 0.0f;
-            // P (bf16) in shared memory as the K-major, 128-byte-swizzled A
-            // operand of O += P V: panel h holds keys 64h..64h+63, row r at
-            // r * 128 bytes, 16-byte chunk c (keys 8c..8c+7) at c ^ (r & 7).
-            // A and B take the one buffer in turn, in the order A(0), B(0),
-            // A(1), B(1), ... (a block past its last tile drops out): a
-            // hand-off waits for the O += P V of the hand-off before it.
-            // That one is at most one phase ahead of what this warpgroup
-            // has already seen on its barrier, so a parity wait is exact.
-            uint8_t *prow = smem + kOffP + row * 128;
-            int prev_x = -1, prev_j = -1;
-            if (x == 0) {
-                if (j >= 1) {
-                    prev_j = j - 1;
-                    prev_x = j - 1 < nB ? 1 : 0;
+            // P_x is free once the O += P V of tile j - 1 has completed.
+            if (j > 0 && !pv_seen) {
+                if (!wait_warp(bar_pv(x), (uint32_t)(j - 1) & 1u, abort_flag, status)) {
+                    ok = false;
+                    break;
                 }
-            } else if (j < nA) {
-                prev_x = 0;
-                prev_j = j;
-            } else if (j >= 1) {
-                prev_x = 1;
-                prev_j = j - 1;
+                tc_fence_after();
             }
-            uint32_t pk[64];  // P of keys 2u, 2u+1 in pk[u]
-            // The exponent arguments come from the packed fp32x2 FMA (the
-            // same rounded fma per element as the scalar form, half the
-            // issues); the four running sums stay scalar adds.
+            // P (bf16) into tensor memory, keys 2u and 2u+1 in column u of
+            // P_x, the layout of the A operand of O += P V.  Half h (keys
+            // 64h .. 64h+63) is stored and released as soon as it is
+            // computed.  The exponent arguments come from the packed fp32x2
+            // FMA (the same rounded fma per element as the scalar form, half
+            // the issues); the four running sums stay scalar adds.
             const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(neg_m, neg_m);
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int u = 0; u < 64; u += 2) {
-                const int c = 2 * u;
-                const float2 x01 = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, nm2);
-                const float2 x23 = __ffma2_rn(make_float2(s[c + 2], s[c + 3]), sc2, nm2);
-                const float2 p01 = make_float2(ex2(x01.x), ex2(x01.y));
-                const float2 p23 = make_float2(ex2(x23.x), ex2(x23.y));
-                ls[0] += p01.x;
-                ls[1] += p01.y;
-                ls[2] += p23.x;
-                ls[3] += p23.y;
-                pk[u] = pack_bf16(p01.x, p01.y);
-                pk[u + 1] = pack_bf16(p23.x, p23.y);
-            }
-            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-            // Hand P over half by half: half h waits for the previous
-            // hand-off's O += P_h V_h, is stored, and is released to the MMA
-            // warp (after the proxy fence that orders the generic-proxy
-            // stores before the tensor core's reads; the first release also
-            // orders any O rescale before the next O += P V).
+            uint32_t pk[64];  // P of keys 2u, 2u+1 in pk[u]
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                if (prev_x >= 0) {
-                    p_free = wait_warp(bar_ph(prev_x, h), (uint32_t)prev_j & 1u, abort_flag, status);
-                    if (!p_free) break;
-                }
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(prow + h * kPanelBytes + ((c ^ (row & 7)) << 4)) =
-                        make_uint4(pk[32 * h + 4 * c], pk[32 * h + 4 * c + 1],
-                                   pk[32 * h + 4 * c + 2], pk[32 * h + 4 * c + 3]);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                if (h == 0) tc_fence_before();
+                for (int u = 32 * h; u < 32 * h + 32; u += 2) {
+                    const int c = 2 * u;
+                    const float2 x01 = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, nm2);
+                    const float2 x23 = __ffma2_rn(make_float2(s[c + 2], s[c + 3]), sc2, nm2);
+                    const float2 p01 = make_float2(ex2(x01.x), ex2(x01.y));
+                    const float2 p23 = make_float2(ex2(x23.x), ex2(x23.y));
+                    ls[0] += p01.x;
+                    ls[1] += p01.y;
+                    ls[2] += p23.x;
+                    ls[3] += p23.y;
+                    pk[u] = pack_bf16(p01.x, p01.y);
+                    pk[u + 1] = pack_bf16(p23.x, p23.y);
+                }
+                // The store completes (wait::st) before the release; the
+                // first release also orders any O rescale before the next
+                // O += P V.
+                tmem_st32(tmem + lane_base + colP + 32 * h, pk + 32 * h);
+                tmem_wait_st();
+                tc_fence_before();
                 mbar_arrive(bar_p(x, h));
             }
-            if (prev_x >= 0 && !p_free) {
-                ok = false;
-                break;
-            }
+            l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         }
 
         // ---- epilogue: O / l -> bf16, LSE
