@@ -15,16 +15,21 @@
 // device address (on the host it names a stand-in), so the first call on
 // each device, with that device current, looks the address up once with
 // cudaGetSymbolAddress and caches it; that first call should be made
-// before any stream capture starts.  All calls share the arena: calls
-// whose work overlaps on the GPU (different streams, or different host
-// threads) race on it and must be serialised by the caller.  Every byte a
-// call reads from the arena is written earlier in the same call, so no
-// clearing is needed.
+// before any stream capture starts.  The cache entry remembers the unique
+// id of the CUDA context it was taken in (cuCtxGetId): a call made in
+// another context (a non-primary one, or a new primary context after
+// cudaDeviceReset, where the module may be loaded at another address)
+// looks the address up again instead of using a stale one.  All calls
+// share the arena: calls whose work overlaps on the GPU (different
+// streams, or different host threads) race on it and must be serialised
+// by the caller.  Every byte a call reads from the arena is written
+// earlier in the same call, so no clearing is needed.
 #include <cmath>
 #include <cstddef>
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
@@ -41,9 +46,41 @@ constexpr int kMaxDevices = 64;
 __device__ __align__(256) unsigned char g_arena[kArenaBytes];
 
 std::mutex g_setup_mutex;
-void *g_arena_addr[kMaxDevices];  // device address of g_arena, per device
+struct ArenaEntry {
+    unsigned long long ctx_id;  // unique id of the context the address belongs to
+    void *addr;                 // device address of g_arena in that context
+};
+ArenaEntry g_arena_cache[kMaxDevices];
 
-// Device address of the arena on the current device (looked up once).
+// Unique id of the calling thread's current CUDA context, or 0 when none
+// is current yet.  The driver entry points are looked up through the
+// runtime, so the library keeps loading on hosts without a driver.
+int current_context_id(unsigned long long *id) {
+    using GetCurrent = CUresult (*)(CUcontext *);
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    if (!get_current || !get_id) {
+        void *a = nullptr, *b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+            qa != cudaDriverEntryPointSuccess || qb != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return SPARSTAR_ECUDA;
+        }
+        get_current = reinterpret_cast<GetCurrent>(a);
+        get_id = reinterpret_cast<GetId>(b);
+    }
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return SPARSTAR_ECUDA;
+    *id = 0;
+    if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return SPARSTAR_ECUDA;
+    return SPARSTAR_OK;
+}
+
+// Device address of the arena on the current device, in the current
+// context (looked up once per device and context).
 int arena_address(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -52,15 +89,25 @@ int arena_address(void **out) {
     }
     if (dev < 0 || dev >= kMaxDevices) return SPARSTAR_ENODEV;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_arena_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_arena) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return SPARSTAR_ECUDA;
-        }
-        g_arena_addr[dev] = p;
+    unsigned long long id = 0;
+    if (int rc = current_context_id(&id)) return rc;
+    ArenaEntry &entry = g_arena_cache[dev];
+    if (id != 0 && entry.addr && entry.ctx_id == id) {
+        *out = entry.addr;
+        return SPARSTAR_OK;
     }
-    *out = g_arena_addr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_arena) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return SPARSTAR_ECUDA;
+    }
+    // The lookup makes the device's primary context current when none was.
+    if (id == 0) {
+        if (int rc = current_context_id(&id)) return rc;
+    }
+    entry.ctx_id = id;
+    entry.addr = p;
+    *out = p;
     return SPARSTAR_OK;
 }
 

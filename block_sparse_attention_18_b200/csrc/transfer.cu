@@ -166,8 +166,12 @@ cudaError_t launch_transfer_lists(const int32_t *src_idx, const int32_t *src_cnt
     // A row is a chain of dependent loads (count, list, bitmap), so up to
     // eight CTAs per SM keep enough rows in flight; the map (a few integer
     // divisions per thread) is cheap to rebuild per CTA.
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
     int64_t ctas = ceil_div(rows, kWarpsPerCta);
-    if (ctas > 148 * 8) ctas = 148 * 8;
+    if (ctas > (int64_t)sms * 8) ctas = (int64_t)sms * 8;
     transfer_kernel<<<(unsigned)ctas, kWarpsPerCta * 32, smem, stream>>>(
         src_idx, src_cnt, src_max_sel, ly, rows, dst_idx, dst_cnt, dst_max_sel, words);
     return cudaGetLastError();

@@ -207,7 +207,11 @@ int sparstar_forward(const void *q, const void *k, const void *v, int dtype, int
  *     59 MB); larger calls return SPARSTAR_ESIZE and launch nothing.
  *   - The first call on each device looks the arena's address up
  *     (cudaGetSymbolAddress) with that device current and caches it; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture.  The cached address is
+ *     tied to the CUDA context it was taken in: a call in another context
+ *     (a non-primary context, or the new primary context after
+ *     cudaDeviceReset) looks it up again, so that call too should come
+ *     before any capture.
  *   - All calls share the arena.  Calls whose GPU work overlaps (other
  *     streams, other host threads) race on it; serialise them.
  * The caller still owns q, k, v, out, lse and status.  Errors are those of
