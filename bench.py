@@ -196,54 +196,65 @@ def max_over_ranks(value: float, world: int, device) -> float:
 
 # --------------------------------------------------------------- CPU oracle
 
-def oracle_sample_step(orc, w, qn, kn, vn, head: int, n_rows: int, seed: int) -> float:
-    """Time the oracle on a bounded sample of one step: the fp32 selection
-    of one head (pool Q, pool K, score, select) and fp64 attention on
-    ``n_rows`` of that head's query rows.  Returns the projected time of a
-    full step in seconds (selection x heads, attention x rows / n_rows)."""
+def oracle_band_step(orc, w, qn, kn, vn, head: int, band: int, n_blocks: int):
+    """One bounded unit of the whole path on the oracle: for one head and
+    the ``n_blocks`` query blocks starting at block ``band``, the fp32
+    selection (pool Q of those blocks, pool K, score, select) and the fp64
+    attention of every one of their query rows.  Returns (seconds, attention
+    FLOPs of the unit): both measured on the same unit, nothing projected."""
     sl = slice(head, head + 1)
-    qh = np.ascontiguousarray(qn[:, sl])
+    r0 = band * 128
+    r1 = min(w.Lq, r0 + n_blocks * 128)
+    qh = np.ascontiguousarray(qn[:, sl, r0:r1])
     kh = np.ascontiguousarray(kn[:, sl])
     vh = np.ascontiguousarray(vn[:, sl])
     t0 = time.perf_counter()
     _, _, _, idx, cnt = orc.run_selection(qh, kh, w.text, w.image_ref, w.density)
-    t_sel = time.perf_counter() - t0
-    rows = np.sort(np.random.default_rng(seed).choice(w.Lq, size=min(n_rows, w.Lq), replace=False))
-    t1 = time.perf_counter()
-    orc.attn_rows_f64(qh, kh, vh, idx, cnt, rows.astype(np.int64))
-    t_att = time.perf_counter() - t1
+    orc.attn_rows_f64(qh, kh, vh, idx, cnt, np.arange(r1 - r0, dtype=np.int64))
+    dt = time.perf_counter() - t0
+    return dt, attention_flops(idx, cnt, r1 - r0, w.Lk, w.D)
+
+
+def _bands(w, n_units: int, n_blocks: int, seed: int):
+    """Seeded (head, first query block) pairs; the first unit holds the
+    last (possibly partial) query block."""
+    rng = np.random.default_rng(seed)
     heads = w.B * w.H
-    return heads * (t_sel + t_att * (w.Lq / len(rows)))
+    first = max(0, w.nQB - n_blocks)
+    out = [(heads - 1, first)]
+    while len(out) < n_units:
+        out.append((int(rng.integers(0, heads)), int(rng.integers(0, first + 1))))
+    return out
 
 
-def oracle_flops(orc, w, qn, kn) -> float:
-    """Algorithmic FLOPs of one full step from the oracle's own selection."""
-    _, _, _, idx, cnt = orc.run_selection(qn, kn, w.text, w.image_ref, w.density)
-    return attention_flops(idx, cnt, w.Lq, w.Lk, w.D)
-
-
-def cpu_baseline(w, qn, kn, vn, flops_step: float, budget_s: float = 15.0, n_rows: int = 4096):
-    """The oracle, as it stands, on this host's cores, on a bounded sample."""
+def cpu_baseline(w, qn, kn, vn, budget_s: float = 15.0, n_blocks: int = 2):
+    """The oracle, as it stands, on this host's cores, on a bounded sample:
+    whole-path units (one head, ``n_blocks`` query blocks) until the time
+    budget is spent.  value = attention FLOPs of the units / their time."""
     import oracle as orc
     orc.lib()
     t_start = time.perf_counter()
-    times, heads = [], []
-    h = 0
-    while len(times) < 2 or (time.perf_counter() - t_start < budget_s and h < w.B * w.H):
-        times.append(oracle_sample_step(orc, w, qn, kn, vn, h, n_rows, seed=h))
-        heads.append(h)
-        h += 1
-    step_s = statistics.mean(times)
-    return {"value": flops_step / step_s / 1e12, "unit": UNIT, "cores": orc.num_threads(),
+    secs, flops, units = 0.0, 0.0, []
+    for head, band in _bands(w, 10 ** 6, n_blocks, seed=7):
+        dt, f = oracle_band_step(orc, w, qn, kn, vn, head, band, n_blocks)
+        secs += dt
+        flops += f
+        units.append((head, band))
+        if time.perf_counter() - t_start > budget_s and len(units) >= 2:
+            break
+    return {"value": flops / secs / 1e12, "unit": UNIT, "cores": orc.num_threads(),
             "kind": "oracle",
-            "sample": ("fp32 selection of heads %s and fp64 attention on %d random query rows of "
-                       "each; time projected to the full step (x%d heads, x%d/%d rows): %.1f s "
-                       "per full step" % (heads, n_rows, w.B * w.H, w.Lq, n_rows, step_s)),
+            "sample": ("%d units of the whole path (fp32 selection, then fp64 attention of every "
+                       "row), each one head x %d query blocks (%d query rows): %.3g attention "
+                       "FLOP in %.2f s; measured, not projected" % (
+                           len(units), n_blocks, n_blocks * 128, flops, secs)),
             "wall_s": time.perf_counter() - t_start}
 
 
 def run_reference(args, world, rank):
-    """The comparison arm: the CPU oracle timed on this host's cores."""
+    """The comparison arm: the CPU oracle timed on this host's cores.  Each
+    step is one bounded unit of the whole path (one head, a band of query
+    blocks); value = attention FLOPs of the timed units / their time."""
     if rank != 0:
         return
     import oracle as orc
@@ -251,24 +262,26 @@ def run_reference(args, world, rank):
     w = bench_workload(args)
     q, k, v = synth.generate(w)
     qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
-    flops = oracle_flops(orc, w, qn, kn)
-    n_rows = args.ref_rows
-    for s in range(args.warmup):
-        oracle_sample_step(orc, w, qn, kn, vn, s % (w.B * w.H), n_rows, seed=1000 + s)
-    times = [oracle_sample_step(orc, w, qn, kn, vn, s % (w.B * w.H), n_rows, seed=s)
-             for s in range(args.steps)]
-    step_s = statistics.mean(times)
-    value = flops / step_s / 1e12
+    nb = args.ref_blocks
+    units = _bands(w, args.warmup + args.steps, nb, seed=11)
+    for head, band in units[:args.warmup]:
+        oracle_band_step(orc, w, qn, kn, vn, head, band, nb)
+    secs, flops = 0.0, 0.0
+    for head, band in units[args.warmup:]:
+        dt, f = oracle_band_step(orc, w, qn, kn, vn, head, band, nb)
+        secs += dt
+        flops += f
+    value = flops / secs / 1e12
+    sample = ("each step: one head x %d query blocks (%d rows) of the workload through the whole "
+              "path (fp32 selection, fp64 attention of every row); %.3g attention FLOP per step "
+              "on average; measured, not projected" % (nb, nb * 128, flops / args.steps))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle",
-                         "cores": orc.num_threads(),
-                         "sample": "each step: fp32 selection of one head and fp64 attention on "
-                                   "%d random query rows of it, projected to the full step "
-                                   "(x%d heads, x%d/%d rows)" % (n_rows, w.B * w.H, w.Lq, n_rows)},
+                         "cores": orc.num_threads(), "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -311,6 +324,14 @@ def front_end_summary(w, per, peaks, clocks):
         out["score_select"] = {"ms": ms, "fp32_tflops": tf, "bound": "alu",
                                "peak_fp32_tflops": fp32_peak, "frac": tf / fp32_peak,
                                "s_bytes_kept_on_chip": s_bytes}
+        # pool and score as one pair against HBM: the algorithmic bytes of
+        # the two steps (Q, K read and means written; means read and S
+        # written) over the time of the two fused launches.
+        pair_bytes = pool_bytes + (w.nQB + w.nKB) * w.D * 4 * bh + s_bytes
+        pair_ms = pool_ms + ms
+        pair_gbs = pair_bytes / (pair_ms * 1e-3) / 1e9
+        out["pool_score"] = {"ms": pair_ms, "bytes": pair_bytes, "gbs": pair_gbs,
+                             "frac_of_hbm": pair_gbs / peaks["hbm_gbs"]}
     else:
         score_bytes = (w.nQB + w.nKB) * w.D * 4 * bh + s_bytes
         out["score"] = {"ms": per["score"], "bytes": score_bytes,
@@ -528,10 +549,92 @@ def run_gpu(args, world, rank, local):
         line["retained_mass"] = mass
     if reuse is not None:
         line["reuse_across_scales"] = reuse
+    if world == 1 and args.per_workload:
+        line["per_workload"] = per_workload(sp, device, stream, peaks)
     if world == 1 and not args.no_cpu_baseline:
         qn, kn, vn = (synth.as_numpy(t) for t in (q, k, v))
-        line["cpu_baseline"] = cpu_baseline(w, qn, kn, vn, flops)
+        line["cpu_baseline"] = cpu_baseline(w, qn, kn, vn)
     print(json.dumps(line), flush=True)
+
+
+def per_workload(sp, device, stream, peaks, steps=10, warmup=3):
+    """Every workload of the synthetic suite through the fused chain (pool
+    Q+K, score+select, attention): ``steps`` steps captured in one CUDA
+    graph and replayed once, per-kernel CUDA events inside.  Workloads whose
+    inputs fit in L2 get an L2 flush (a write of twice the L2 size) before
+    each step, outside the timed kernels."""
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device=device)
+    res = {}
+    for name, w in synth.WORKLOADS.items():
+        q, k, v = synth.generate(w)
+        qd, kd, vd = q.to(device), k.to(device), v.to(device)
+        del q, k, v
+        ws = sp.Workspace(w.B, w.H, w.D, w.text, w.image_ref, w.ref, w.cur, w.density, device,
+                          scores=False)
+        out = torch.empty_like(qd)
+        lse = torch.empty(w.B, w.H, w.Lq, device=device, dtype=torch.float32)
+        status = torch.zeros(1, dtype=torch.int32, device=device)
+        tau = sp.default_tau(w.D)
+        in_bytes = sum(t.numel() * t.element_size() for t in (qd, kd, vd))
+        do_flush = in_bytes < 2 * l2
+
+        def step(st, ev=None):
+            if do_flush:
+                flush.fill_(1.0)
+            if ev: ev[0].record(st)
+            sp.sparstar_block_pool_qk(qd, kd, ws.qbar, ws.kbar, stream=st)
+            if ev: ev[1].record(st)
+            sp.sparstar_score_select(ws.qbar, ws.kbar, ws.n_forced, w.density, tau,
+                                     kv_idx=ws.kv_idx, kv_cnt=ws.kv_cnt, stream=st)
+            if ev: ev[2].record(st)
+            sp.sparstar_attn_fwd(qd, kd, vd, ws.kv_idx, ws.kv_cnt, tau, out, lse, status,
+                                 stream=st)
+            if ev: ev[3].record(st)
+
+        for _ in range(warmup):
+            step(stream)
+        torch.cuda.synchronize(device)
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+               for _ in range(steps)]
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap), torch.cuda.graph(graph, stream=cap):
+            for i in range(steps):
+                step(cap, evs[i])
+        stream.wait_stream(cap)
+        graph.replay()
+        torch.cuda.synchronize(device)
+        with ClockSampler(device.index) as clk:
+            clk.wait_first()
+            h0 = time.monotonic()
+            graph.replay()
+            torch.cuda.synchronize(device)
+            h1 = time.monotonic()
+            time.sleep(0.06)
+            clk.window = (h0, h1 + 0.05)
+        del graph
+        if int(status.item()) != 0:
+            raise SystemExit("%s: attention kernel status %#x" % (name, int(status.item())))
+        kms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
+        flops = attention_flops(ws.kv_idx.cpu().numpy(), ws.kv_cnt.cpu().numpy(), w.Lq, w.Lk,
+                                w.D)
+        attn_tf = flops / (kms[2] * 1e-3) / 1e12
+        fe = front_end_summary(w, {"pool_qk": kms[0], "score_select": kms[1]}, peaks,
+                               clk.summary())
+        res[name] = {
+            "step_ms": sum(kms), "pool_qk_ms": kms[0], "score_select_ms": kms[1],
+            "attn_ms": kms[2], "attn_tflops": attn_tf,
+            "attn_frac_of_measured_burst": attn_tf / peaks["bf16_tflops"] if w.dtype == "bf16"
+            else None,
+            "pool_score_frac_of_hbm": fe["pool_score"]["frac_of_hbm"],
+            "front_end_share_pct": 100 * (kms[0] + kms[1]) / sum(kms),
+            "sm_mhz": clk.summary().get("sm_mhz"), "l2_flushed": do_flush,
+        }
+        del qd, kd, vd, ws, out, lse
+        torch.cuda.empty_cache()
+    return res
 
 
 def mass_rows(w, per_head, device, seed=0):
@@ -711,8 +814,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--seed", type=int, default=None,
                     help="seed of the synthetic inputs (default: the workload's own)")
-    ap.add_argument("--ref-rows", type=int, default=256,
-                    help="query rows per sampled step of the reference arm")
+    ap.add_argument("--ref-blocks", type=int, default=2,
+                    help="query blocks (of one head) per step of the reference arm")
     ap.add_argument("--chain", choices=["fused", "separate"], default="fused",
                     help="timed step: pool_qk + score_select + attn (fused) or the five "
                          "separate calls; the other chain is timed eagerly beside it")
@@ -725,6 +828,8 @@ def main(argv=None):
                     help="skip the mask-reuse diagnostic (lists of the previous scale carried "
                          "to this one)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", dest="per_workload", action="store_false",
+                    help="skip the table of every workload (single GPU only)")
     ap.add_argument("--no-dense", dest="dense", action="store_false",
                     help="skip the dense comparison point (density 1 and torch SDPA)")
     args = ap.parse_args(argv)

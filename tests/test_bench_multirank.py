@@ -53,7 +53,7 @@ def _ref_worker(rank, world, port, results):
     calls = []
     try:
         class Args:
-            workload, steps, warmup, ref_rows = "tiny", 1, 3, 16
+            workload, steps, warmup, ref_blocks = "tiny", 1, 3, 2
         import io
         import contextlib
         buf = io.StringIO()
