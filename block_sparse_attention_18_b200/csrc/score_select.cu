@@ -505,6 +505,280 @@ score_select_tiled_kernel(const __grid_constant__ CUtensorMap tmK, const float *
                 kv_cnt, max_sel);
 }
 
+// ------------------------------------------------------- column scores
+//
+// The column kernel (nKB <= 256 * kMaxNc), 512 threads: thread t owns key
+// columns t % 256 + 256 c (c < NC) and the 8 query rows 8 (t / 256) .. +7 of
+// the CTA's 16, so it accumulates 8 x NC outputs.  Key means arrive by TMA as
+// 16-wide d-chunks of every key column (NC boxes of 16 floats x 256 rows,
+// 64-byte rows, 64-byte swizzle) through a two-slot ring; the query means
+// sit in shared memory and every read of them is a warp-wide broadcast.  Per
+// 4 values of d a thread issues NC key loads (one wavefront per 8 lanes) and
+// 8 query loads for 32 NC FMAs.  Each output takes its FMAs in ascending d
+// from acc = +0, so the scores are bit for bit those of the other kernels.
+// When the last chunk is multiplied the ring is idle and holds the score
+// rows.
+//
+// Its selection (select_rows_bits) keeps one row per warp in registers:
+// lane l holds the row's columns l * kpl .. l * kpl + kpl - 1 (kpl a
+// multiple of 4 whose quarter is odd, so the lanes' 16-byte loads spread
+// over all banks), non-candidates as key 0 (every score's key is above 0).
+// The threshold T, the k-th largest key, comes from a bitwise search below
+// the row's common leading bits, each step one count over the registers
+// and a warp sum; then every lane counts its keys > T and == T, and warp
+// prefix sums place them: all keys > T and the first k - count(> T) keys
+// == T in ascending column order (ties to the lower block index).  No
+// histogram, no shared-memory list: the same lists as select_rows.
+
+constexpr int kMaxNc = 6;          // up to 1536 key blocks
+constexpr int kColRing = 2;        // ring depth, in chunks
+constexpr int kColChunkD = 16;     // d values per chunk (64-byte rows)
+constexpr int kColThreads = 512;   // two row groups of 256 column threads
+constexpr int kColWarps = kColThreads / 32;
+constexpr int kGroupRows = kRows / 2;
+
+// Lane segment length: the smallest multiple of 4 with an odd quarter that
+// covers nKB with 32 lanes.
+constexpr int seg_len(int nKB) {
+    int q = (nKB + 127) / 128;  // quarter of ceil(nKB / 32), rounded up
+    return 4 * (q | 1);
+}
+constexpr int kpl_max(int NC) { return seg_len(256 * NC); }
+constexpr int64_t col_stride(int NC) { return 32LL * kpl_max(NC); }
+constexpr int64_t col_slot_bytes(int NC) { return (int64_t)NC * 256 * kColChunkD * 4; }
+constexpr int64_t col_rows_bytes(int NC) { return 4LL * kRows * col_stride(NC); }
+constexpr int64_t col_region_bytes(int NC) {
+    return kColRing * col_slot_bytes(NC) > col_rows_bytes(NC) ? kColRing * col_slot_bytes(NC)
+                                                              : col_rows_bytes(NC);
+}
+template <int D, int NC>
+constexpr int64_t col_smem() {
+    return 1024 + col_region_bytes(NC) + (int64_t)kRows * D * 4 + 8 * kColRing;
+}
+
+// Warp-wide exclusive prefix sum of v; *total receives the sum.
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t &total) {
+    const int lane = threadIdx.x & 31;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    total = __shfl_sync(0xffffffffu, incl, 31);
+    return incl - v;
+}
+
+// Selection of the CTA's rows from register-held segments (see above).
+// Same contract as select_rows, with NW warps: warp w takes rows w, w + NW,
+// ...; `failed` rows get an empty list.
+template <int KPL, int NW>
+__device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, int64_t bh,
+                                 int64_t i0, int64_t nQB, int nKB, int nF, int k, bool failed,
+                                 int32_t *__restrict__ kv_idx, int32_t *__restrict__ kv_cnt,
+                                 int64_t max_sel) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int C = nKB - nF;
+    const int c0 = lane * kpl;  // first column of this lane's segment
+    for (int r = warp; r < kRows; r += NW) {
+        const int64_t i = i0 + r;
+        if (i >= nQB) break;  // warp-uniform; later rows are further out
+        const int64_t grow = bh * nQB + i;
+        int32_t *out = kv_idx + grow * max_sel;
+        int written = 0;
+        if (!failed) {
+            for (int f = lane; f < nF; f += 32) out[f] = f;
+            written = nF;
+        }
+        if (!failed && k > 0) {
+            // Candidate keys of this lane's segment; other columns read as 0.
+            uint32_t v[KPL];
+            const uint32_t *seg = srows + r * stride + c0;
+            const int lo_c = nF - c0, hi_c = nKB - c0;
+#pragma unroll
+            for (int g = 0; g < KPL / 4; ++g) {
+                uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
+                if (4 * g < kpl) w4 = *reinterpret_cast<const uint4 *>(seg + 4 * g);
+                v[4 * g] = (4 * g >= lo_c && 4 * g < hi_c) ? w4.x : 0u;
+                v[4 * g + 1] = (4 * g + 1 >= lo_c && 4 * g + 1 < hi_c) ? w4.y : 0u;
+                v[4 * g + 2] = (4 * g + 2 >= lo_c && 4 * g + 2 < hi_c) ? w4.z : 0u;
+                v[4 * g + 3] = (4 * g + 3 >= lo_c && 4 * g + 3 < hi_c) ? w4.w : 0u;
+            }
+            uint32_t T = 0u;  // k == C: every candidate key is > 0, all taken
+            if (k < C) {
+                uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    if (v[e]) kmin = min(kmin, v[e]);
+                    kmax = max(kmax, v[e]);
+                }
+                kmin = __reduce_min_sync(0xffffffffu, kmin);
+                kmax = __reduce_max_sync(0xffffffffu, kmax);
+                // The k-th largest key: the largest t with count(key >= t) >= k,
+                // built bit by bit below the common leading bits of kmin, kmax.
+                const int p = __clz(kmin ^ kmax);
+                uint32_t prefix = p == 32 ? kmin : (p == 0 ? 0u : kmin & ~(0xffffffffu >> p));
+                for (int bit = 31 - p; bit >= 0; --bit) {
+                    const uint32_t cand = prefix | (1u << bit);
+                    uint32_t n = 0u;
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) n += v[e] >= cand ? 1u : 0u;
+                    if (__reduce_add_sync(0xffffffffu, n) >= (uint32_t)k) prefix = cand;
+                }
+                T = prefix;
+            }
+            uint32_t n_gt = 0u, n_eq = 0u;
+#pragma unroll
+            for (int e = 0; e < KPL; ++e) {
+                n_gt += v[e] > T ? 1u : 0u;
+                n_eq += v[e] == T ? 1u : 0u;
+            }
+            uint32_t gt_total;
+            warp_excl_scan(n_gt, gt_total);
+            const uint32_t need = (uint32_t)k - gt_total;  // keys == T still to take
+            // Ties go to the lower block index: the first `need` keys == T in
+            // ascending column order, i.e. lane order then register order.
+            uint32_t eq_total;
+            const uint32_t eq_before = warp_excl_scan(n_eq, eq_total);
+            const uint32_t eq_take = need > eq_before ? min(need - eq_before, n_eq) : 0u;
+            uint32_t taken;
+            uint32_t dst = (uint32_t)nF + warp_excl_scan(n_gt + eq_take, taken);
+            uint32_t eq_seen = 0u;
+#pragma unroll
+            for (int e = 0; e < KPL; ++e) {
+                const bool eq = v[e] == T;
+                if (v[e] > T || (eq && eq_seen < eq_take)) out[dst++] = c0 + e;
+                eq_seen += eq ? 1u : 0u;
+            }
+            written = nF + (int)taken;
+        }
+        for (int64_t s2 = written + lane; s2 < max_sel; s2 += 32) out[s2] = -1;
+        if (lane == 0) kv_cnt[grow] = failed ? 0 : nF + k;
+    }
+}
+
+template <int D, int NC>
+__global__ void __launch_bounds__(kColThreads, 1)
+score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *__restrict__ qbar,
+                         int64_t nQB, int nKB, int kpl, int64_t n_qtiles, float tau, int nF,
+                         int k, int32_t *__restrict__ kv_idx, int32_t *__restrict__ kv_cnt,
+                         int64_t max_sel, int32_t *status) {
+    constexpr int kChunks = D / kColChunkD;
+    constexpr int kSlotBytes = (int)col_slot_bytes(NC);
+    constexpr int kStride = (int)col_stride(NC);
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char *ks = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    float *qs = reinterpret_cast<float *>(ks + col_region_bytes(NC));     // [kRows][D]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(qs + kRows * D);
+    uint32_t *srows = reinterpret_cast<uint32_t *>(ks);  // after scoring: [kRows][kStride]
+
+    const int tid = threadIdx.x;
+    const int grp = tid / 256, tc = tid % 256;  // row group (rows 8 grp ..), column thread
+    const int64_t bh = blockIdx.x / n_qtiles;
+    const int64_t i0 = (blockIdx.x - bh * n_qtiles) * kRows;
+    auto bar = [&](int sl) { return smem_addr(bars + sl); };
+    auto issue = [&](int step) {  // thread 0 only: chunk `step` of every column
+        const int slot = step % kColRing;
+        mbar_expect_tx(bar(slot), kSlotBytes);
+#pragma unroll
+        for (int b = 0; b < NC; ++b)
+            tma_load_3d(smem_addr(ks + slot * kSlotBytes + b * 256 * kColChunkD * 4), &tmK,
+                        bar(slot), step * kColChunkD, b * 256, (int)bh);
+    };
+
+    int issued = 0;  // meaningful in thread 0
+    if (tid == 0) {
+        for (int sl = 0; sl < kColRing; ++sl) mbar_init(bar(sl), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (; issued < kColRing && issued < kChunks; ++issued) issue(issued);
+    }
+    for (int idx = tid; idx < kRows * (D / 4); idx += kColThreads) {
+        const int row = idx / (D / 4), v = idx % (D / 4);
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i0 + row < nQB)
+            a = *reinterpret_cast<const float4 *>(qbar + ((bh * nQB) + i0 + row) * D + 4 * v);
+        *reinterpret_cast<float4 *>(qs + row * D + 4 * v) = a;
+    }
+    __syncthreads();
+
+    // This thread: rows 8 grp .. 8 grp + 7, columns tc + 256 c.  Its column's
+    // 64-byte row in a box holds d chunks of 16 bytes, chunk h stored at
+    // h ^ ((tc >> 1) & 3) (the 64-byte swizzle), which spreads a warp's
+    // loads of one chunk over all banks.
+    const float *qg = qs + grp * kGroupRows * D;
+    const int swz = (tc >> 1) & 3;
+    float acc[NC][kGroupRows];
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int r = 0; r < kGroupRows; ++r) acc[c][r] = 0.0f;
+    bool failed = false;
+    int step = 0;
+#pragma unroll 1
+    for (; step < kChunks; ++step) {
+        const int slot = step % kColRing;
+        const bool ok = mbar_wait(bar(slot), (uint32_t)(step / kColRing) & 1u);
+        const unsigned char *kc = ks + slot * kSlotBytes + tc * kColChunkD * 4;
+#pragma unroll
+        for (int h = 0; h < kColChunkD / 4; ++h) {  // d = 16 step + 4h .. + 3
+            float4 kv[NC], qv[kGroupRows];
+#pragma unroll
+            for (int c = 0; c < NC; ++c)
+                kv[c] = *reinterpret_cast<const float4 *>(kc + c * 256 * kColChunkD * 4 +
+                                                          ((h ^ swz) << 4));
+#pragma unroll
+            for (int r = 0; r < kGroupRows; ++r)
+                qv[r] = *reinterpret_cast<const float4 *>(qg + r * D + kColChunkD * step + 4 * h);
+#pragma unroll
+            for (int r = 0; r < kGroupRows; ++r)
+#pragma unroll
+                for (int c = 0; c < NC; ++c) acc[c][r] = __fmaf_rn(qv[r].x, kv[c].x, acc[c][r]);
+#pragma unroll
+            for (int r = 0; r < kGroupRows; ++r)
+#pragma unroll
+                for (int c = 0; c < NC; ++c) acc[c][r] = __fmaf_rn(qv[r].y, kv[c].y, acc[c][r]);
+#pragma unroll
+            for (int r = 0; r < kGroupRows; ++r)
+#pragma unroll
+                for (int c = 0; c < NC; ++c) acc[c][r] = __fmaf_rn(qv[r].z, kv[c].z, acc[c][r]);
+#pragma unroll
+            for (int r = 0; r < kGroupRows; ++r)
+#pragma unroll
+                for (int c = 0; c < NC; ++c) acc[c][r] = __fmaf_rn(qv[r].w, kv[c].w, acc[c][r]);
+        }
+        // Every thread is done with this slot (and learns of any timeout).
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        if (tid == 0 && issued < kChunks) issue(issued++);
+    }
+    if (failed) {
+        if (tid == 0) {
+            for (int st = step; st < issued; ++st)
+                mbar_wait(bar(st % kColRing), (uint32_t)(st / kColRing) & 1u);
+            if (status) atomicOr(status, SPARSTAR_STATUS_TIMEOUT);
+        }
+        __syncthreads();
+    } else {
+        // Keys into the score rows, over the ring: every thread is past the
+        // last chunk, and no copy is in flight.
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const int j = tc + 256 * c;
+            if (j < nKB) {
+#pragma unroll
+                for (int rr = 0; rr < kGroupRows; ++rr)
+                    srows[(grp * kGroupRows + rr) * kStride + j] =
+                        order_key(__fmul_rn(acc[c][rr], tau));
+            }
+        }
+        __syncthreads();
+    }
+    select_rows_bits<kpl_max(NC), kColWarps>(srows, kStride, kpl, bh, i0, nQB, nKB, nF, k,
+                                             failed, kv_idx, kv_cnt, max_sel);
+}
+
 // ----------------------------------------------------------- wide scores
 
 constexpr int kWTile = 128;      // key blocks per staged tile
@@ -654,6 +928,53 @@ bool encode_kbar(CUtensorMap *map, const float *kbar, int64_t BH, int64_t nKB, i
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// kbar [BH, nKB, D] fp32 as a 3-D tensor; box = 16 floats x 256 rows x 1
+// (64-byte rows), 64-byte swizzle.  Rows past nKB read as zero.
+bool encode_kbar_cols(CUtensorMap *map, const float *kbar, int64_t BH, int64_t nKB, int D) {
+    auto fn = get_encoder();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)nKB, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)nKB * D * 4};
+    const cuuint32_t box[3] = {(cuuint32_t)kColChunkD, 256, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(kbar), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int NC>
+cudaError_t launch_cols_nc(const float *qbar, const float *kbar, int64_t BH, int64_t nQB,
+                           int64_t nKB, float tau, int64_t nF, int64_t k, int32_t *kv_idx,
+                           int32_t *kv_cnt, int64_t max_sel, int32_t *status, cudaStream_t s) {
+    CUtensorMap tm;
+    if (!encode_kbar_cols(&tm, kbar, BH, nKB, D)) return cudaErrorInvalidValue;
+    constexpr int64_t smem = col_smem<D, NC>();
+    static_assert(smem <= kMaxSmem, "column kernel shared memory");
+    cudaError_t e = cudaFuncSetAttribute(score_select_cols_kernel<D, NC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t n_qtiles = ceil_div(nQB, kRows);
+    score_select_cols_kernel<D, NC><<<(unsigned)(BH * n_qtiles), kColThreads, (size_t)smem, s>>>(
+        tm, qbar, nQB, (int)nKB, seg_len((int)nKB), n_qtiles, tau, (int)nF, (int)k, kv_idx,
+        kv_cnt, max_sel, status);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_cols(const float *qbar, const float *kbar, int64_t BH, int64_t nQB,
+                        int64_t nKB, float tau, int64_t nF, int64_t k, int32_t *kv_idx,
+                        int32_t *kv_cnt, int64_t max_sel, int32_t *status, cudaStream_t s) {
+    switch (ceil_div(nKB, 256)) {
+    case 1: return launch_cols_nc<D, 1>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt, max_sel, status, s);
+    case 2: return launch_cols_nc<D, 2>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt, max_sel, status, s);
+    case 3: return launch_cols_nc<D, 3>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt, max_sel, status, s);
+    case 4: return launch_cols_nc<D, 4>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt, max_sel, status, s);
+    case 5: return launch_cols_nc<D, 5>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt, max_sel, status, s);
+    case 6: return launch_cols_nc<D, 6>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt, max_sel, status, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 template <int D>
 cudaError_t launch_tiled(const float *qbar, const float *kbar, int64_t BH, int64_t nQB,
                          int64_t nKB, float tau, int64_t nF, int64_t k, int32_t *kv_idx,
@@ -705,6 +1026,11 @@ cudaError_t launch_score_select(const float *qbar, const float *kbar, int64_t BH
                                 int64_t nKB, int D, float tau, int64_t nF, int64_t k,
                                 int32_t *kv_idx, int32_t *kv_cnt, int64_t max_sel,
                                 int32_t *status, cudaStream_t stream) {
+    if (nKB <= 256 * kMaxNc)
+        return D == 128 ? launch_cols<128>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt,
+                                           max_sel, status, stream)
+                        : launch_cols<64>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt,
+                                          max_sel, status, stream);
     if (nKB <= kTiledMaxNkb)
         return D == 128 ? launch_tiled<128>(qbar, kbar, BH, nQB, nKB, tau, nF, k, kv_idx, kv_cnt,
                                             max_sel, status, stream)

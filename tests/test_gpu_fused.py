@@ -72,6 +72,18 @@ EDGE = {
     "f32_d128": dict(H=2, dtype="f32", text=256, ref=2000, cur=2100, density=0.25),
     # Clip-1 layout: a forced prefix that ends inside a block
     "clip1": dict(H=2, text=512, image_ref=3600, ref=2000, cur=2000, density=0.1875),
+    # the column kernel at its key-column boundaries: nKB = 256 (one column
+    # per thread), 257 (two), 1536 (its largest), then 1537 (the TMA-tiled
+    # kernel's first)
+    "cols_nkb256": dict(H=2, text=128, ref=127 * 128, cur=128 * 128, density=0.15),
+    "cols_nkb257": dict(H=2, text=128, ref=127 * 128 + 1, cur=128 * 128, density=0.15),
+    "cols_max": dict(H=1, text=512, ref=1536 * 128 - 512 - 10 * 128, cur=10 * 128,
+                     density=0.1),
+    "tiled_min": dict(H=1, text=512, ref=1536 * 128 - 512 - 10 * 128 + 1, cur=10 * 128,
+                      density=0.1),
+    # the column kernel with crowded buckets (lists longer than 64 keys)
+    "cols_one_bucket": dict(H=2, text=256, ref=40000, cur=38000, density=0.3,
+                            offset_std=1e-3),
     # the TMA-tiled kernel's largest nKB (1664), then the first wide one (1665)
     "tiled_max": dict(H=1, text=512, ref=1650 * 128, cur=10 * 128, density=0.1),
     "wide_min": dict(H=1, text=512, ref=1650 * 128 + 1, cur=10 * 128, density=0.1),
