@@ -525,10 +525,12 @@ score_select_tiled_kernel(const __grid_constant__ CUtensorMap tmK, const float *
 // over all banks), non-candidates as key 0 (every score's key is above 0).
 // The threshold T, the k-th largest key, comes from a bitwise search below
 // the row's common leading bits, each step one count over the registers
-// and a warp sum; then every lane counts its keys > T and == T, and warp
-// prefix sums place them: all keys > T and the first k - count(> T) keys
-// == T in ascending column order (ties to the lower block index).  No
-// histogram, no shared-memory list: the same lists as select_rows.
+// and a warp sum, that narrows a window [prefix, prefix + 2^(b+1)) holding
+// T; once the window holds at most 64 keys they are compacted into a
+// per-warp list and T is ranked there (list_threshold).  Then every lane
+// counts its keys > T and == T, and warp prefix sums place them: all keys
+// > T and the first k - count(> T) keys == T in ascending column order
+// (ties to the lower block index).  The same lists as select_rows.
 
 constexpr int kMaxNc = 6;          // up to 1536 key blocks
 constexpr int kColRing = 2;        // ring depth, in chunks
@@ -551,6 +553,9 @@ constexpr int64_t col_region_bytes(int NC) {
     return kColRing * col_slot_bytes(NC) > col_rows_bytes(NC) ? kColRing * col_slot_bytes(NC)
                                                               : col_rows_bytes(NC);
 }
+static_assert(kColRing * col_slot_bytes(1) >= col_rows_bytes(1) + kColWarps * 64 * 4 &&
+                  kColRing * col_slot_bytes(6) >= col_rows_bytes(6) + kColWarps * 64 * 4,
+              "the ring region holds the score rows and the per-warp window lists");
 template <int D, int NC>
 constexpr int64_t col_smem() {
     return 1024 + col_region_bytes(NC) + (int64_t)kRows * D * 4 + 8 * kColRing;
@@ -572,12 +577,15 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t &total) 
 // Selection of the CTA's rows from register-held segments (see above).
 // Same contract as select_rows, with NW warps: warp w takes rows w, w + NW,
 // ...; `failed` rows get an empty list.
+constexpr uint32_t kWindowList = 64;  // window size at which the search moves to a list
+
 template <int KPL, int NW>
-__device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, int64_t bh,
-                                 int64_t i0, int64_t nQB, int nKB, int nF, int k, bool failed,
-                                 int32_t *__restrict__ kv_idx, int32_t *__restrict__ kv_cnt,
-                                 int64_t max_sel) {
+__device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, uint32_t *scratch,
+                                 int64_t bh, int64_t i0, int64_t nQB, int nKB, int nF, int k,
+                                 bool failed, int32_t *__restrict__ kv_idx,
+                                 int32_t *__restrict__ kv_cnt, int64_t max_sel) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t *list = scratch + warp * kWindowList;
     const int C = nKB - nF;
     const int c0 = lane * kpl;  // first column of this lane's segment
     for (int r = warp; r < kRows; r += NW) {
@@ -616,16 +624,50 @@ __device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, int
                 kmax = __reduce_max_sync(0xffffffffu, kmax);
                 // The k-th largest key: the largest t with count(key >= t) >= k,
                 // built bit by bit below the common leading bits of kmin, kmax.
+                // The window [prefix, prefix + 2^(bit+1)) holds it, with
+                // count(>= prefix) = lo >= k and count(>= window end) = hi < k.
                 const int p = __clz(kmin ^ kmax);
                 uint32_t prefix = p == 32 ? kmin : (p == 0 ? 0u : kmin & ~(0xffffffffu >> p));
-                for (int bit = 31 - p; bit >= 0; --bit) {
+                uint32_t lo = (uint32_t)C, hi = 0u;
+                int bit = 31 - p;
+                for (; bit >= 0 && lo - hi > kWindowList; --bit) {
                     const uint32_t cand = prefix | (1u << bit);
-                    uint32_t n = 0u;
+                    uint32_t n0 = 0u, n1 = 0u;
 #pragma unroll
-                    for (int e = 0; e < KPL; ++e) n += v[e] >= cand ? 1u : 0u;
-                    if (__reduce_add_sync(0xffffffffu, n) >= (uint32_t)k) prefix = cand;
+                    for (int e = 0; e < KPL; e += 2) {
+                        n0 += v[e] >= cand ? 1u : 0u;
+                        n1 += (e + 1 < KPL && v[e + 1] >= cand) ? 1u : 0u;
+                    }
+                    const uint32_t c = __reduce_add_sync(0xffffffffu, n0 + n1);
+                    if (c >= (uint32_t)k) {
+                        prefix = cand;
+                        lo = c;
+                    } else {
+                        hi = c;
+                    }
                 }
-                T = prefix;
+                if (bit < 0) {
+                    T = prefix;  // the window is one key value
+                } else {
+                    // The window's lo - hi keys into the list, then the
+                    // (k - hi)-th largest of them.  Non-candidates are key 0,
+                    // below every candidate: the window starts at 1 at least.
+                    const uint32_t start = prefix > 1u ? prefix : 1u;
+                    const uint64_t end = (uint64_t)prefix + (2ull << bit);
+                    uint32_t n_in = 0u;
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e)
+                        n_in += (v[e] >= start && (uint64_t)v[e] < end) ? 1u : 0u;
+                    uint32_t m;
+                    uint32_t pos = warp_excl_scan(n_in, m);
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e)
+                        if (v[e] >= start && (uint64_t)v[e] < end) list[pos++] = v[e];
+                    __syncwarp();
+                    uint32_t need_in;
+                    list_threshold(list, (int)m, (uint32_t)k - hi, T, need_in);
+                    __syncwarp();  // list reads done before the next row reuses it
+                }
             }
             uint32_t n_gt = 0u, n_eq = 0u;
 #pragma unroll
@@ -775,8 +817,9 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
         }
         __syncthreads();
     }
-    select_rows_bits<kpl_max(NC), kColWarps>(srows, kStride, kpl, bh, i0, nQB, nKB, nF, k,
-                                             failed, kv_idx, kv_cnt, max_sel);
+    select_rows_bits<kpl_max(NC), kColWarps>(srows, kStride, kpl,
+                                             srows + kRows * kStride, bh, i0, nQB, nKB, nF,
+                                             k, failed, kv_idx, kv_cnt, max_sel);
 }
 
 // ----------------------------------------------------------- wide scores
