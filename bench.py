@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # SHA-256 of the kernel source it was taken on; reported only while the
 # source is unchanged.
 ATTN_TRAFFIC = {
-    "source_sha256": "86fc765e3339fad23cbae11967a36cb4492735509520144ab9235526a8213179",
-    "bytes_per_launch": 3505765888 + 292825344,  # largest workload, one launch
+    "source_sha256": "e0af731107adf0fe4e9531a4dc2aaa9a1c32fdc93728c7cd175d924d95dc16d1",
+    "bytes_per_launch": 3580000000 + 290000000,  # largest workload, one launch (3.58 GB + 290 MB)
 }
 
 
