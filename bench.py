@@ -16,6 +16,7 @@ step is a bounded sample of the same workload (one head's selection and a
 set of its query rows in fp64), projected to the full step.
 """
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -799,10 +800,19 @@ def dense_comparison(sp, w, qd, kd, vd, tau, sparse_attn_ms, stream, reps=3):
 
 def bench_workload(args):
     """The workload named on the command line, with --seed replacing its
-    seed when given (the synthetic inputs are drawn from that seed)."""
+    seed when given (the synthetic inputs are drawn from that seed) and
+    --heads its head count (a smaller launch of the same shapes, for
+    profiling)."""
     w = synth.WORKLOADS[args.workload]
     seed = getattr(args, "seed", None)
-    return w if seed is None else synth.with_seed(w, seed)
+    if seed is not None:
+        w = synth.with_seed(w, seed)
+    heads = getattr(args, "heads", None)
+    if heads is not None:
+        if heads < 1:
+            raise SystemExit("--heads must be at least 1")
+        w = dataclasses.replace(w, H=heads)
+    return w
 
 
 def main(argv=None):
@@ -814,6 +824,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=list(synth.WORKLOADS))
     ap.add_argument("--seed", type=int, default=None,
                     help="seed of the synthetic inputs (default: the workload's own)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="head count replacing the workload's own (smaller launches of the "
+                         "same per-head shapes, for profiling)")
     ap.add_argument("--ref-blocks", type=int, default=2,
                     help="query blocks (of one head) per step of the reference arm")
     ap.add_argument("--chain", choices=["fused", "separate"], default="fused",
