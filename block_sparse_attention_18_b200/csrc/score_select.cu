@@ -509,13 +509,16 @@ score_select_tiled_kernel(const __grid_constant__ CUtensorMap tmK, const float *
 //
 // The column kernel (nKB <= 256 * kMaxNc), 512 threads: thread t owns key
 // columns t % 256 + 256 c (c < NC) and the 8 query rows 8 (t / 256) .. +7 of
-// the CTA's 16, so it accumulates 8 x NC outputs.  Key means arrive by TMA as
-// 16-wide d-chunks of every key column (NC boxes of 16 floats x 256 rows,
-// 64-byte rows, 64-byte swizzle) through a two-slot ring; the query means
-// sit in shared memory and every read of them is a warp-wide broadcast.  Per
-// 4 values of d a thread issues NC key loads (one wavefront per 8 lanes) and
-// 8 query loads for 32 NC FMAs.  Each output takes its FMAs in ascending d
-// from acc = +0, so the scores are bit for bit those of the other kernels.
+// the CTA's 16, so it accumulates 8 x NC outputs as 4 x NC float2 row pairs
+// advanced by the packed fp32x2 FMA (two independent round-to-nearest fmas
+// per instruction).  Key means arrive by TMA as 16-wide d-chunks of every
+// key column (NC boxes of 16 floats x 256 rows, 64-byte rows, 64-byte
+// swizzle) through a two-slot ring; the query means sit in shared memory,
+// row pairs interleaved, and every read of them is a warp-wide broadcast.
+// Per 4 values of d a thread issues NC key loads (one wavefront per 8 lanes)
+// and 8 query loads for 16 NC packed FMAs.  Each output takes its FMAs in
+// ascending d from acc = +0, so the scores are bit for bit those of the
+// other kernels.
 // When the last chunk is multiplied the ring is idle and holds the score
 // rows.
 //
@@ -739,7 +742,14 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
         float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
         if (i0 + row < nQB)
             a = *reinterpret_cast<const float4 *>(qbar + ((bh * nQB) + i0 + row) * D + 4 * v);
-        *reinterpret_cast<float4 *>(qs + row * D + 4 * v) = a;
+        // Row pairs interleaved: float2 (row 2P, row 2P + 1) of group g at d
+        // is qs[((4 g + P) D + d) 2 ..].
+        float *dst = qs + (((row / kGroupRows) * (kGroupRows / 2) + (row % kGroupRows) / 2) * D +
+                           4 * v) * 2 + (row % 2);
+        dst[0] = a.x;
+        dst[2] = a.y;
+        dst[4] = a.z;
+        dst[6] = a.w;
     }
     __syncthreads();
 
@@ -749,11 +759,11 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
     // loads of one chunk over all banks.
     const float *qg = qs + grp * kGroupRows * D;
     const int swz = (tc >> 1) & 3;
-    float acc[NC][kGroupRows];
+    float2 acc[NC][kGroupRows / 2];  // (row 2P, row 2P + 1) of column c
 #pragma unroll
     for (int c = 0; c < NC; ++c)
 #pragma unroll
-        for (int r = 0; r < kGroupRows; ++r) acc[c][r] = 0.0f;
+        for (int r = 0; r < kGroupRows / 2; ++r) acc[c][r] = make_float2(0.0f, 0.0f);
     bool failed = false;
     int step = 0;
 #pragma unroll 1
@@ -763,30 +773,44 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
         const unsigned char *kc = ks + slot * kSlotBytes + tc * kColChunkD * 4;
 #pragma unroll
         for (int h = 0; h < kColChunkD / 4; ++h) {  // d = 16 step + 4h .. + 3
-            float4 kv[NC], qv[kGroupRows];
+            // Per d: one packed fp32x2 FMA per (column, row pair), the key
+            // mean in both halves; each half is the same round-to-nearest
+            // fma as the scalar form.
+            float4 kv[NC], qv[kGroupRows / 2][2];
 #pragma unroll
             for (int c = 0; c < NC; ++c)
                 kv[c] = *reinterpret_cast<const float4 *>(kc + c * 256 * kColChunkD * 4 +
                                                           ((h ^ swz) << 4));
 #pragma unroll
-            for (int r = 0; r < kGroupRows; ++r)
-                qv[r] = *reinterpret_cast<const float4 *>(qg + r * D + kColChunkD * step + 4 * h);
+            for (int pr = 0; pr < kGroupRows / 2; ++pr)
 #pragma unroll
-            for (int r = 0; r < kGroupRows; ++r)
+                for (int e = 0; e < 2; ++e)
+                    qv[pr][e] = *reinterpret_cast<const float4 *>(
+                        qg + (pr * D + kColChunkD * step + 4 * h + 2 * e) * 2);
 #pragma unroll
-                for (int c = 0; c < NC; ++c) acc[c][r] = __fmaf_rn(qv[r].x, kv[c].x, acc[c][r]);
+            for (int pr = 0; pr < kGroupRows / 2; ++pr)
 #pragma unroll
-            for (int r = 0; r < kGroupRows; ++r)
+                for (int c = 0; c < NC; ++c)
+                    acc[c][pr] = __ffma2_rn(make_float2(qv[pr][0].x, qv[pr][0].y),
+                                            make_float2(kv[c].x, kv[c].x), acc[c][pr]);
 #pragma unroll
-                for (int c = 0; c < NC; ++c) acc[c][r] = __fmaf_rn(qv[r].y, kv[c].y, acc[c][r]);
+            for (int pr = 0; pr < kGroupRows / 2; ++pr)
 #pragma unroll
-            for (int r = 0; r < kGroupRows; ++r)
+                for (int c = 0; c < NC; ++c)
+                    acc[c][pr] = __ffma2_rn(make_float2(qv[pr][0].z, qv[pr][0].w),
+                                            make_float2(kv[c].y, kv[c].y), acc[c][pr]);
 #pragma unroll
-                for (int c = 0; c < NC; ++c) acc[c][r] = __fmaf_rn(qv[r].z, kv[c].z, acc[c][r]);
+            for (int pr = 0; pr < kGroupRows / 2; ++pr)
 #pragma unroll
-            for (int r = 0; r < kGroupRows; ++r)
+                for (int c = 0; c < NC; ++c)
+                    acc[c][pr] = __ffma2_rn(make_float2(qv[pr][1].x, qv[pr][1].y),
+                                            make_float2(kv[c].z, kv[c].z), acc[c][pr]);
 #pragma unroll
-                for (int c = 0; c < NC; ++c) acc[c][r] = __fmaf_rn(qv[r].w, kv[c].w, acc[c][r]);
+            for (int pr = 0; pr < kGroupRows / 2; ++pr)
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+                    acc[c][pr] = __ffma2_rn(make_float2(qv[pr][1].z, qv[pr][1].w),
+                                            make_float2(kv[c].w, kv[c].w), acc[c][pr]);
         }
         // Every thread is done with this slot (and learns of any timeout).
         if (__syncthreads_or(!ok)) {
@@ -810,9 +834,12 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
             const int j = tc + 256 * c;
             if (j < nKB) {
 #pragma unroll
-                for (int rr = 0; rr < kGroupRows; ++rr)
-                    srows[(grp * kGroupRows + rr) * kStride + j] =
-                        order_key(__fmul_rn(acc[c][rr], tau));
+                for (int pr = 0; pr < kGroupRows / 2; ++pr) {
+                    srows[(grp * kGroupRows + 2 * pr) * kStride + j] =
+                        order_key(__fmul_rn(acc[c][pr].x, tau));
+                    srows[(grp * kGroupRows + 2 * pr + 1) * kStride + j] =
+                        order_key(__fmul_rn(acc[c][pr].y, tau));
+                }
             }
         }
         __syncthreads();

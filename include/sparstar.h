@@ -251,10 +251,11 @@ int sparstar_block_pool_qk(const void *q, const void *k, int dtype, int64_t B, i
  * The score rows of 16 query blocks must fit in one CTA's shared memory:
  * nKB <= sparstar_score_select_max_nkb(D) (2432 for D = 128, 2944 for
  * D = 64, i.e. about 311k / 377k keys), else SPARSTAR_ESIZE and nothing is
- * launched; the separate calls have no such limit.  Up to nKB = 1664 the
- * key tiles arrive by TMA into a 4 x 4-per-thread product; larger nKB use a
- * register-staged tiling that needs less shared memory per key block.
- * Other errors as for the separate calls.
+ * launched; the separate calls have no such limit.  Up to nKB = 1536 the
+ * key means arrive by TMA as d-chunks of every key column (8 rows x up to 6
+ * columns per thread); up to 1664 as 256-key tiles (4 x 4 per thread);
+ * larger nKB use a register-staged tiling that needs less shared memory per
+ * key block.  Other errors as for the separate calls.
  */
 int sparstar_score_select(const float *qbar, const float *kbar, int64_t B, int64_t H,
                           int64_t nQB, int64_t nKB, int64_t D, float tau,
