@@ -516,7 +516,8 @@ score_select_tiled_kernel(const __grid_constant__ CUtensorMap tmK, const float *
 // swizzle) through a two-slot ring; the query means sit in shared memory,
 // row pairs interleaved, and every read of them is a warp-wide broadcast.
 // Per 4 values of d a thread issues NC key loads (one wavefront per 8 lanes)
-// and 8 query loads for 16 NC packed FMAs.  Each output takes its FMAs in
+// and 8 query loads for 16 NC packed FMAs; a warp whose columns in the last
+// block all lie past nKB skips that block.  Each output takes its FMAs in
 // ascending d from acc = +0, so the scores are bit for bit those of the
 // other kernels.
 // When the last chunk is multiplied the ring is idle and holds the score
@@ -525,7 +526,8 @@ score_select_tiled_kernel(const __grid_constant__ CUtensorMap tmK, const float *
 // Its selection (select_rows_bits) keeps one row per warp in registers:
 // lane l holds the row's columns l * kpl .. l * kpl + kpl - 1 (kpl a
 // multiple of 4 whose quarter is odd, so the lanes' 16-byte loads spread
-// over all banks), non-candidates as key 0 (every score's key is above 0).
+// over all banks; the selection is compiled for both values kpl takes at a
+// given NC), non-candidates as key 0 (every score's key is above 0).
 // The threshold T, the k-th largest key, comes from a bitwise search below
 // the row's common leading bits, each step one count over the registers
 // and a warp sum, that narrows a window [prefix, prefix + 2^(b+1)) holding
@@ -617,12 +619,16 @@ __device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, uin
             }
             uint32_t T = 0u;  // k == C: every candidate key is > 0, all taken
             if (k < C) {
-                uint32_t kmin = 0xffffffffu, kmax = 0u;
+                // Four partial minima and maxima (shorter dependency chains).
+                uint32_t mn[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+                uint32_t mx[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                 for (int e = 0; e < KPL; ++e) {
-                    if (v[e]) kmin = min(kmin, v[e]);
-                    kmax = max(kmax, v[e]);
+                    if (v[e]) mn[e & 3] = min(mn[e & 3], v[e]);
+                    mx[e & 3] = max(mx[e & 3], v[e]);
                 }
+                uint32_t kmin = min(min(mn[0], mn[1]), min(mn[2], mn[3]));
+                uint32_t kmax = max(max(mx[0], mx[1]), max(mx[2], mx[3]));
                 kmin = __reduce_min_sync(0xffffffffu, kmin);
                 kmax = __reduce_max_sync(0xffffffffu, kmax);
                 // The k-th largest key: the largest t with count(key >= t) >= k,
@@ -635,13 +641,11 @@ __device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, uin
                 int bit = 31 - p;
                 for (; bit >= 0 && lo - hi > kWindowList; --bit) {
                     const uint32_t cand = prefix | (1u << bit);
-                    uint32_t n0 = 0u, n1 = 0u;
+                    uint32_t nc[4] = {0u, 0u, 0u, 0u};  // KPL is a multiple of 4
 #pragma unroll
-                    for (int e = 0; e < KPL; e += 2) {
-                        n0 += v[e] >= cand ? 1u : 0u;
-                        n1 += (e + 1 < KPL && v[e + 1] >= cand) ? 1u : 0u;
-                    }
-                    const uint32_t c = __reduce_add_sync(0xffffffffu, n0 + n1);
+                    for (int e = 0; e < KPL; ++e) nc[e & 3] += v[e] >= cand ? 1u : 0u;
+                    const uint32_t c =
+                        __reduce_add_sync(0xffffffffu, (nc[0] + nc[1]) + (nc[2] + nc[3]));
                     if (c >= (uint32_t)k) {
                         prefix = cand;
                         lo = c;
@@ -702,6 +706,53 @@ __device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, uin
     }
 }
 
+// One 16-wide d-chunk of the column kernel's product for the first NCC of
+// the thread's NC column blocks: per d, one packed fp32x2 FMA per (column,
+// row pair), the key mean in both halves; each half is the same
+// round-to-nearest fma as the scalar form, in ascending d.
+template <int D, int NCC, int NC>
+__device__ __forceinline__ void col_chunk_fma(const unsigned char *kc, const float *qg, int step,
+                                              int swz, float2 (&acc)[NC][kGroupRows / 2]) {
+#pragma unroll
+    for (int h = 0; h < kColChunkD / 4; ++h) {  // d = 16 step + 4h .. + 3
+        float4 kv[NCC > 0 ? NCC : 1], qv[kGroupRows / 2][2];
+#pragma unroll
+        for (int c = 0; c < NCC; ++c)
+            kv[c] = *reinterpret_cast<const float4 *>(kc + c * 256 * kColChunkD * 4 +
+                                                      ((h ^ swz) << 4));
+#pragma unroll
+        for (int pr = 0; pr < kGroupRows / 2; ++pr)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                qv[pr][e] = *reinterpret_cast<const float4 *>(
+                    qg + (pr * D + kColChunkD * step + 4 * h + 2 * e) * 2);
+#pragma unroll
+        for (int pr = 0; pr < kGroupRows / 2; ++pr)
+#pragma unroll
+            for (int c = 0; c < NCC; ++c)
+                acc[c][pr] = __ffma2_rn(make_float2(qv[pr][0].x, qv[pr][0].y), make_float2(kv[c].x, kv[c].x),
+                                        acc[c][pr]);
+#pragma unroll
+        for (int pr = 0; pr < kGroupRows / 2; ++pr)
+#pragma unroll
+            for (int c = 0; c < NCC; ++c)
+                acc[c][pr] = __ffma2_rn(make_float2(qv[pr][0].z, qv[pr][0].w), make_float2(kv[c].y, kv[c].y),
+                                        acc[c][pr]);
+#pragma unroll
+        for (int pr = 0; pr < kGroupRows / 2; ++pr)
+#pragma unroll
+            for (int c = 0; c < NCC; ++c)
+                acc[c][pr] = __ffma2_rn(make_float2(qv[pr][1].x, qv[pr][1].y), make_float2(kv[c].z, kv[c].z),
+                                        acc[c][pr]);
+#pragma unroll
+        for (int pr = 0; pr < kGroupRows / 2; ++pr)
+#pragma unroll
+            for (int c = 0; c < NCC; ++c)
+                acc[c][pr] = __ffma2_rn(make_float2(qv[pr][1].z, qv[pr][1].w), make_float2(kv[c].w, kv[c].w),
+                                        acc[c][pr]);
+    }
+}
+
 template <int D, int NC>
 __global__ void __launch_bounds__(kColThreads, 1)
 score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *__restrict__ qbar,
@@ -759,6 +810,9 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
     // loads of one chunk over all banks.
     const float *qg = qs + grp * kGroupRows * D;
     const int swz = (tc >> 1) & 3;
+    // A warp whose lowest column in the last column block is past nKB skips
+    // that block (its outputs are never written).
+    const bool last_live = (tc & ~31) + 256 * (NC - 1) < nKB;
     float2 acc[NC][kGroupRows / 2];  // (row 2P, row 2P + 1) of column c
 #pragma unroll
     for (int c = 0; c < NC; ++c)
@@ -771,47 +825,10 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
         const int slot = step % kColRing;
         const bool ok = mbar_wait(bar(slot), (uint32_t)(step / kColRing) & 1u);
         const unsigned char *kc = ks + slot * kSlotBytes + tc * kColChunkD * 4;
-#pragma unroll
-        for (int h = 0; h < kColChunkD / 4; ++h) {  // d = 16 step + 4h .. + 3
-            // Per d: one packed fp32x2 FMA per (column, row pair), the key
-            // mean in both halves; each half is the same round-to-nearest
-            // fma as the scalar form.
-            float4 kv[NC], qv[kGroupRows / 2][2];
-#pragma unroll
-            for (int c = 0; c < NC; ++c)
-                kv[c] = *reinterpret_cast<const float4 *>(kc + c * 256 * kColChunkD * 4 +
-                                                          ((h ^ swz) << 4));
-#pragma unroll
-            for (int pr = 0; pr < kGroupRows / 2; ++pr)
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-                    qv[pr][e] = *reinterpret_cast<const float4 *>(
-                        qg + (pr * D + kColChunkD * step + 4 * h + 2 * e) * 2);
-#pragma unroll
-            for (int pr = 0; pr < kGroupRows / 2; ++pr)
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-                    acc[c][pr] = __ffma2_rn(make_float2(qv[pr][0].x, qv[pr][0].y),
-                                            make_float2(kv[c].x, kv[c].x), acc[c][pr]);
-#pragma unroll
-            for (int pr = 0; pr < kGroupRows / 2; ++pr)
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-                    acc[c][pr] = __ffma2_rn(make_float2(qv[pr][0].z, qv[pr][0].w),
-                                            make_float2(kv[c].y, kv[c].y), acc[c][pr]);
-#pragma unroll
-            for (int pr = 0; pr < kGroupRows / 2; ++pr)
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-                    acc[c][pr] = __ffma2_rn(make_float2(qv[pr][1].x, qv[pr][1].y),
-                                            make_float2(kv[c].z, kv[c].z), acc[c][pr]);
-#pragma unroll
-            for (int pr = 0; pr < kGroupRows / 2; ++pr)
-#pragma unroll
-                for (int c = 0; c < NC; ++c)
-                    acc[c][pr] = __ffma2_rn(make_float2(qv[pr][1].z, qv[pr][1].w),
-                                            make_float2(kv[c].w, kv[c].w), acc[c][pr]);
-        }
+        if (last_live)
+            col_chunk_fma<D, NC, NC>(kc, qg, step, swz, acc);
+        else
+            col_chunk_fma<D, NC - 1, NC>(kc, qg, step, swz, acc);
         // Every thread is done with this slot (and learns of any timeout).
         if (__syncthreads_or(!ok)) {
             failed = true;
@@ -844,9 +861,16 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
         }
         __syncthreads();
     }
-    select_rows_bits<kpl_max(NC), kColWarps>(srows, kStride, kpl,
-                                             srows + kRows * kStride, bh, i0, nQB, nKB, nF,
-                                             k, failed, kv_idx, kv_cnt, max_sel);
+    // kpl is kpl_max(NC) or kpl_max(NC) - 8 (seg_len of nKB in (256 (NC - 1), 256 NC]);
+    // the selection loops run over exactly kpl registers.
+    if (kpl == kpl_max(NC))
+        select_rows_bits<kpl_max(NC), kColWarps>(srows, kStride, kpl, srows + kRows * kStride,
+                                                 bh, i0, nQB, nKB, nF, k, failed, kv_idx, kv_cnt,
+                                                 max_sel);
+    else
+        select_rows_bits<kpl_max(NC) - 8, kColWarps>(srows, kStride, kpl,
+                                                     srows + kRows * kStride, bh, i0, nQB, nKB,
+                                                     nF, k, failed, kv_idx, kv_cnt, max_sel);
 }
 
 // ----------------------------------------------------------- wide scores
