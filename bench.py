@@ -301,6 +301,14 @@ def workload_config(w, world):
 
 # --------------------------------------------------------------- GPU arm
 
+def fp32_peak_tflops(clocks):
+    """FP32 FMA roofline: SMs x 128 lanes x 2 flops x the maximum SM clock."""
+    mhz = clocks.get("sm_max_mhz") or 1965.0
+    sms = torch.cuda.get_device_properties(0).multi_processor_count \
+        if torch.cuda.is_available() else 148
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
 def front_end_summary(w, per, peaks, clocks):
     """Rooflines of the selection kernels.  Pooling is HBM-bound: bytes = the
     Q and K reads + the mean writes.  The score is a fixed-order fp32 FMA
@@ -317,8 +325,7 @@ def front_end_summary(w, per, peaks, clocks):
     pool_gbs = pool_bytes / (pool_ms * 1e-3) / 1e9
     out = {"pool": {"ms": pool_ms, "bytes": pool_bytes, "gbs": pool_gbs,
                     "frac_of_hbm": pool_gbs / peaks["hbm_gbs"], "bound": "hbm"}}
-    mhz = clocks.get("sm_max_mhz") or 1965.0
-    fp32_peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    fp32_peak = fp32_peak_tflops(clocks)
     if "score_select" in per:
         ms = per["score_select"]
         tf = score_flops / (ms * 1e-3) / 1e12
@@ -629,6 +636,11 @@ def per_workload(sp, device, stream, peaks, steps=10, warmup=3):
             "attn_ms": kms[2], "attn_tflops": attn_tf,
             "attn_frac_of_measured_burst": attn_tf / peaks["bf16_tflops"] if w.dtype == "bf16"
             else None,
+            # fp32 inputs run the fp32 SIMT kernel: its roofline is the FP32 FMA rate.
+            "attn_roofline": "bf16 tensor (measured burst)" if w.dtype == "bf16"
+            else "fp32 FMA (SMs x 128 lanes x 2 x max clock)",
+            "attn_frac_of_roofline": attn_tf / (peaks["bf16_tflops"] if w.dtype == "bf16"
+                                                else fp32_peak_tflops(clk.summary())),
             "pool_score_frac_of_hbm": fe["pool_score"]["frac_of_hbm"],
             "front_end_share_pct": 100 * (kms[0] + kms[1]) / sum(kms),
             "sm_mhz": clk.summary().get("sm_mhz"), "l2_flushed": do_flush,
