@@ -295,8 +295,20 @@ def workload_config(w, world):
             "seq_len": w.Lq, "keys": w.Lk, "heads": w.H, "head_dim": w.D, "density": w.density,
             "seed": w.seed,
             "global_batch": w.B * world, "parallelism": "replicas" if world > 1 else "single",
-            "l2": "no flush: inputs (%.2f GB) larger than L2" % (
-                (w.Lq + 2 * w.Lk) * w.H * w.D * (2 if w.dtype == "bf16" else 4) / 1e9)}
+            "l2": l2_note(w)}
+
+
+def l2_note(w):
+    """How the timed region treats L2 (no flush between steps): the note says
+    whether this workload's inputs exceed the L2 or fit in it."""
+    gb = w.B * (w.Lq + 2 * w.Lk) * w.H * w.D * (2 if w.dtype == "bf16" else 4) / 1e9
+    l2 = 126 * 2 ** 20
+    if torch.cuda.is_available():
+        l2 = getattr(torch.cuda.get_device_properties(0), "L2_cache_size", l2) or l2
+    if gb * 1e9 > 2 * l2:
+        return "no flush: inputs (%.2f GB) larger than L2" % gb
+    return ("no flush: inputs (%.3f GB) fit in L2, so the headline figure is L2-warm; the "
+            "per_workload entry of this workload flushes L2 before each step" % gb)
 
 
 # --------------------------------------------------------------- GPU arm
