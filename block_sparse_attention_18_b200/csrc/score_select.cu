@@ -532,10 +532,12 @@ score_select_tiled_kernel(const __grid_constant__ CUtensorMap tmK, const float *
 // the row's common leading bits, each step one count over the registers
 // and a warp sum, that narrows a window [prefix, prefix + 2^(b+1)) holding
 // T; once the window holds at most 64 keys they are compacted into a
-// per-warp list and T is ranked there (list_threshold).  Then every lane
-// counts its keys > T and == T, and warp prefix sums place them: all keys
-// > T and the first k - count(> T) keys == T in ascending column order
-// (ties to the lower block index).  The same lists as select_rows.
+// per-warp list, two keys per lane, and the bitwise search goes on over
+// those registers down to bit 0.  Then every lane counts its keys > T and
+// == T, and a warp prefix sum places them: all keys > T and the first
+// k - count(> T) keys == T in ascending column order (ties to the lower
+// block index; the prefix sum over the ties only runs when there are more
+// keys == T than places).  The same lists as select_rows.
 
 constexpr int kMaxNc = 6;          // up to 1536 key blocks
 constexpr int kColRing = 2;        // ring depth, in chunks
@@ -671,9 +673,19 @@ __device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, uin
                     for (int e = 0; e < KPL; ++e)
                         if (v[e] >= start && (uint64_t)v[e] < end) list[pos++] = v[e];
                     __syncwarp();
-                    uint32_t need_in;
-                    list_threshold(list, (int)m, (uint32_t)k - hi, T, need_in);
+                    // The bitwise search goes on over the list, two keys per
+                    // lane: T = the largest t with count(list >= t) >= k - hi.
+                    const uint32_t a0 = lane < (int)m ? list[lane] : 0u;
+                    const uint32_t a1 = lane + 32 < (int)m ? list[lane + 32] : 0u;
                     __syncwarp();  // list reads done before the next row reuses it
+                    const uint32_t need1 = (uint32_t)k - hi;
+                    for (; bit >= 0; --bit) {
+                        const uint32_t cand = prefix | (1u << bit);
+                        const uint32_t c = __reduce_add_sync(
+                            0xffffffffu, (a0 >= cand ? 1u : 0u) + (a1 >= cand ? 1u : 0u));
+                        if (c >= need1) prefix = cand;
+                    }
+                    T = prefix;
                 }
             }
             uint32_t n_gt = 0u, n_eq = 0u;
@@ -682,14 +694,18 @@ __device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, uin
                 n_gt += v[e] > T ? 1u : 0u;
                 n_eq += v[e] == T ? 1u : 0u;
             }
-            uint32_t gt_total;
-            warp_excl_scan(n_gt, gt_total);
+            const uint32_t gt_total = __reduce_add_sync(0xffffffffu, n_gt);
+            const uint32_t eq_total = __reduce_add_sync(0xffffffffu, n_eq);
             const uint32_t need = (uint32_t)k - gt_total;  // keys == T still to take
             // Ties go to the lower block index: the first `need` keys == T in
             // ascending column order, i.e. lane order then register order.
-            uint32_t eq_total;
-            const uint32_t eq_before = warp_excl_scan(n_eq, eq_total);
-            const uint32_t eq_take = need > eq_before ? min(need - eq_before, n_eq) : 0u;
+            // Without surplus ties (eq_total == need) every key == T is taken.
+            uint32_t eq_take = n_eq;
+            if (eq_total > need) {  // warp-uniform
+                uint32_t tmp;
+                const uint32_t eq_before = warp_excl_scan(n_eq, tmp);
+                eq_take = need > eq_before ? min(need - eq_before, n_eq) : 0u;
+            }
             uint32_t taken;
             uint32_t dst = (uint32_t)nF + warp_excl_scan(n_gt + eq_take, taken);
             uint32_t eq_seen = 0u;
