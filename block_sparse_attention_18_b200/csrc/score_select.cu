@@ -606,18 +606,18 @@ __device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, uin
             written = nF;
         }
         if (!failed && k > 0) {
-            // Candidate keys of this lane's segment; other columns read as 0.
+            // Candidate keys of this lane's segment; the score rows hold 0
+            // for the forced blocks and past nKB, below every candidate key.
             uint32_t v[KPL];
             const uint32_t *seg = srows + r * stride + c0;
-            const int lo_c = nF - c0, hi_c = nKB - c0;
 #pragma unroll
             for (int g = 0; g < KPL / 4; ++g) {
                 uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
                 if (4 * g < kpl) w4 = *reinterpret_cast<const uint4 *>(seg + 4 * g);
-                v[4 * g] = (4 * g >= lo_c && 4 * g < hi_c) ? w4.x : 0u;
-                v[4 * g + 1] = (4 * g + 1 >= lo_c && 4 * g + 1 < hi_c) ? w4.y : 0u;
-                v[4 * g + 2] = (4 * g + 2 >= lo_c && 4 * g + 2 < hi_c) ? w4.z : 0u;
-                v[4 * g + 3] = (4 * g + 3 >= lo_c && 4 * g + 3 < hi_c) ? w4.w : 0u;
+                v[4 * g] = w4.x;
+                v[4 * g + 1] = w4.y;
+                v[4 * g + 2] = w4.z;
+                v[4 * g + 3] = w4.w;
             }
             uint32_t T = 0u;  // k == C: every candidate key is > 0, all taken
             if (k < C) {
@@ -861,19 +861,25 @@ score_select_cols_kernel(const __grid_constant__ CUtensorMap tmK, const float *_
         __syncthreads();
     } else {
         // Keys into the score rows, over the ring: every thread is past the
-        // last chunk, and no copy is in flight.
+        // last chunk, and no copy is in flight.  Forced blocks and columns
+        // past nKB hold key 0 (below every score's key), so the selection
+        // reads its segments without masking.
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             const int j = tc + 256 * c;
-            if (j < nKB) {
+            const bool cand = j >= nF && j < nKB;
 #pragma unroll
-                for (int pr = 0; pr < kGroupRows / 2; ++pr) {
-                    srows[(grp * kGroupRows + 2 * pr) * kStride + j] =
-                        order_key(__fmul_rn(acc[c][pr].x, tau));
-                    srows[(grp * kGroupRows + 2 * pr + 1) * kStride + j] =
-                        order_key(__fmul_rn(acc[c][pr].y, tau));
-                }
+            for (int pr = 0; pr < kGroupRows / 2; ++pr) {
+                srows[(grp * kGroupRows + 2 * pr) * kStride + j] =
+                    cand ? order_key(__fmul_rn(acc[c][pr].x, tau)) : 0u;
+                srows[(grp * kGroupRows + 2 * pr + 1) * kStride + j] =
+                    cand ? order_key(__fmul_rn(acc[c][pr].y, tau)) : 0u;
             }
+        }
+        // Segments may reach past the 256 NC columns (32 kpl > 256 NC).
+        for (int idx = tid; idx < kRows * (32 * kpl - 256 * NC); idx += kColThreads) {
+            const int w = 32 * kpl - 256 * NC;
+            srows[(idx / w) * kStride + 256 * NC + idx % w] = 0u;
         }
         __syncthreads();
     }
