@@ -531,13 +531,15 @@ score_select_tiled_kernel(const __grid_constant__ CUtensorMap tmK, const float *
 // The threshold T, the k-th largest key, comes from a bitwise search below
 // the row's common leading bits, each step one count over the registers
 // and a warp sum, that narrows a window [prefix, prefix + 2^(b+1)) holding
-// T; once the window holds at most 64 keys they are compacted into a
-// per-warp list, two keys per lane, and the bitwise search goes on over
-// those registers down to bit 0.  Then every lane counts its keys > T and
-// == T, and a warp prefix sum places them: all keys > T and the first
-// k - count(> T) keys == T in ascending column order (ties to the lower
-// block index; the prefix sum over the ties only runs when there are more
-// keys == T than places).  The same lists as select_rows.
+// T (on long rows whose keys span several binades, T's binade is found
+// first by galloping from kmax or kmin and bisecting); once the window
+// holds at most 64 keys they are compacted into a per-warp list, two keys
+// per lane, and the bitwise search goes on over those registers down to
+// bit 0.  Then every lane counts its keys > T and == T, and a warp prefix
+// sum places them: all keys > T and the first k - count(> T) keys == T in
+// ascending column order (ties to the lower block index; the prefix sum
+// over the ties only runs when there are more keys == T than places).  The
+// same lists as select_rows.
 
 constexpr int kMaxNc = 6;          // up to 1536 key blocks
 constexpr int kColRing = 2;        // ring depth, in chunks
@@ -637,17 +639,64 @@ __device__ void select_rows_bits(const uint32_t *srows, int stride, int kpl, uin
                 // built bit by bit below the common leading bits of kmin, kmax.
                 // The window [prefix, prefix + 2^(bit+1)) holds it, with
                 // count(>= prefix) = lo >= k and count(>= window end) = hi < k.
+                auto count_ge = [&](uint32_t cand) {  // warp-wide count of keys >= cand
+                    uint32_t nc[4] = {0u, 0u, 0u, 0u};  // KPL is a multiple of 4
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) nc[e & 3] += v[e] >= cand ? 1u : 0u;
+                    return __reduce_add_sync(0xffffffffu, (nc[0] + nc[1]) + (nc[2] + nc[3]));
+                };
                 const int p = __clz(kmin ^ kmax);
                 uint32_t prefix = p == 32 ? kmin : (p == 0 ? 0u : kmin & ~(0xffffffffu >> p));
                 uint32_t lo = (uint32_t)C, hi = 0u;
                 int bit = 31 - p;
+                if (p < 9 && C > 4 * (int)kWindowList) {
+                    // kmin and kmax lie in different binades (the top 9 key bits:
+                    // sign and exponent) and the row is long: find T's binade
+                    // first, galloping from the end nearer to T (from kmax when
+                    // k <= C / 2, else from kmin), then bisecting; counts are of
+                    // keys >= j << 23.  (Short rows reach the 64-key window in a
+                    // few bitwise steps anyway.)
+                    // Invariant: count(>= j << 23) = lo >= k > hi = count(>= jh << 23).
+                    const uint32_t jmin = kmin >> 23, jmax = kmax >> 23;
+                    uint32_t j, jh;
+                    if (2 * (uint32_t)k <= (uint32_t)C) {
+                        j = jmax;
+                        jh = jmax + 1;  // nothing lies above kmax's binade: hi = 0
+                        lo = count_ge(j << 23 > 1u ? j << 23 : 1u);
+                        for (uint32_t d = 1; lo < (uint32_t)k; d <<= 1) {
+                            jh = j;
+                            hi = lo;
+                            j = j > jmin + d ? j - d : jmin;  // all C keys lie >= jmin << 23
+                            lo = count_ge(j << 23 > 1u ? j << 23 : 1u);
+                        }
+                    } else {
+                        j = jmin;  // lo = C
+                        jh = jmin + 1;
+                        hi = count_ge(jh << 23);
+                        for (uint32_t d = 2; hi >= (uint32_t)k; d <<= 1) {
+                            j = jh;
+                            lo = hi;
+                            jh = jh + d < jmax + 1 ? jh + d : jmax + 1;
+                            hi = jh == jmax + 1 ? 0u : count_ge(jh << 23);
+                        }
+                    }
+                    while (jh - j > 1) {
+                        const uint32_t jm = (j + jh) >> 1;
+                        const uint32_t cm = count_ge(jm << 23);
+                        if (cm >= (uint32_t)k) {
+                            j = jm;
+                            lo = cm;
+                        } else {
+                            jh = jm;
+                            hi = cm;
+                        }
+                    }
+                    prefix = j << 23;
+                    bit = 22;  // the window is binade j: [j << 23, (j + 1) << 23)
+                }
                 for (; bit >= 0 && lo - hi > kWindowList; --bit) {
                     const uint32_t cand = prefix | (1u << bit);
-                    uint32_t nc[4] = {0u, 0u, 0u, 0u};  // KPL is a multiple of 4
-#pragma unroll
-                    for (int e = 0; e < KPL; ++e) nc[e & 3] += v[e] >= cand ? 1u : 0u;
-                    const uint32_t c =
-                        __reduce_add_sync(0xffffffffu, (nc[0] + nc[1]) + (nc[2] + nc[3]));
+                    const uint32_t c = count_ge(cand);
                     if (c >= (uint32_t)k) {
                         prefix = cand;
                         lo = c;
