@@ -7,7 +7,9 @@ sparstar_score_select, sparstar_forward_fused) with the oracle.
   tails, query-block counts that are not a multiple of the 16 rows a CTA
   scores, key-block counts at and around the 128-wide staging tile, exact
   ties (duplicated key blocks, all-zero query blocks), k = 1, k = C, C = 0,
-  D = 64, fp32 inputs, and the largest nKB the fused kernel accepts.
+  long rows whose threshold search gallops up from the smallest key or spans
+  many binades, D = 64, fp32 inputs, and the largest nKB the fused kernel
+  accepts.
 - The whole fused chain, eager and replayed from a captured CUDA graph,
   against the oracle's attention on sampled rows.
 """
@@ -84,6 +86,11 @@ EDGE = {
     # the column kernel with crowded buckets (lists longer than 64 keys)
     "cols_one_bucket": dict(H=2, text=256, ref=40000, cur=38000, density=0.3,
                             offset_std=1e-3),
+    # long rows: the threshold's binade found by galloping up from the
+    # smallest key (k > C/2), and scores spread over many binades
+    "cols_gallop_up": dict(H=2, text=256, ref=40000, cur=38000, density=0.8),
+    "cols_wide_range": dict(H=2, text=256, ref=40000, cur=38000, density=0.2,
+                            offset_std=50.0),
     # the TMA-tiled kernel's largest nKB (1664), then the first wide one (1665)
     "tiled_max": dict(H=1, text=512, ref=1650 * 128, cur=10 * 128, density=0.1),
     "wide_min": dict(H=1, text=512, ref=1650 * 128 + 1, cur=10 * 128, density=0.1),
